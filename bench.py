@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the ClusterKV-style recall hot path on B200.
+
+One step = the whole path over one batch of synthetic input: cosine k-means of
+every problem's keys after prefill (strided seeding, T rounds of assign /
+index / update), then one decode step (cluster scoring + budgeted selection,
+sparse attention). Workload: a Llama-2-7B-shaped layer at 32k context (32 KV
+heads, d = 128, C = 400, T = 10, B = 1024, 16 sinks, 64 recent tokens).
+
+Printed metric: keys clustered per second over the whole step (value), with
+decode steps per second measured separately, the roofline of the dominant
+kernel (the tensor-core assignment) and of the decode path, the oracle timed
+on the host cores as a baseline, and an end-to-end number through the public
+C-ABI calls with host buffers.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch under torch.distributed.run: every rank runs the same
+workload on its own GPU (the problems are independent; no collective on the
+data path), and the time is the max over ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from semantic_cluster_recall_b200 import ckv, synth  # noqa: E402
+from semantic_cluster_recall_b200.pipeline import ClusterRecall  # noqa: E402
+
+WORKLOAD = "llama2_layer_32k"
+METRIC = "k-means keys/s (prefill) and sparse-decode steps/s at 32k ctx; % of roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_traffic(name: str):
+    """DRAM bytes per launch of a kernel from a committed ncu summary, or None
+    once the kernel's source has changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)[name]
+        src = os.path.join(ROOT, d["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != d["source_sha256_16"]:
+            return None
+        return float(d["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max over ranks (timing only; no data-path collective)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+
+class Step:
+    """The whole hot path on one batch, through the stage entry points of the C
+    ABI (the same kernels, in the same order, that ckv_cluster runs), with CUDA
+    events around every assignment launch and around the decode step."""
+
+    def __init__(self, w: synth.Workload, dev, stream):
+        self.w, self.dev, self.stream = w, dev, stream
+        self.K, self.V = synth.make_kv(w, device=dev)
+        self.q = synth.make_queries(w, device=dev)
+        self.st = ClusterRecall(w.P, w.G, w.d, w.torch_dtype, w.L_cap, w.S, w.B, w.C, w.N,
+                                w.W, dev, stream=stream)
+        st = self.st
+        self.ws = ckv.workspace(ckv.ckv_cluster_workspace_bytes(w.P, w.N, w.C), dev)
+        st.n_clusters.fill_(w.C)
+        st.tail_begin.fill_(w.L - w.W)
+        st.tail_end.fill_(w.L)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.launches_per_step = 1 + w.T * 5 + 2 + 2
+
+    def run(self, ev_assign=None, ev_decode=None):
+        w, st, K = self.w, self.st, self.K
+        tb, te = w.S, w.L - w.W
+        ckv.ckv_init_centroids(K, K.stride(0), tb, te, w.C, 0, w.C, st.centroids,
+                               st.centroids_hat, st.centroids_lp, stream=self.stream)
+        for t in range(w.T):
+            if ev_assign is not None:
+                ev_assign[t][0].record(self.stream)
+            ckv.ckv_assign(K, K.stride(0), tb, te, st.centroids_hat, w.C, 0, w.C, st.labels, 0,
+                           w.N, stream=self.stream)
+            if ev_assign is not None:
+                ev_assign[t][1].record(self.stream)
+            ckv.ckv_index(st.labels, w.P, tb, te, w.C, 0, w.C, 0, w.N, st.offsets, st.perm,
+                          self.ws, stream=self.stream)
+            ckv.ckv_update(K, K.stride(0), tb, te, w.C, 0, w.C, st.offsets, st.perm, w.N,
+                           st.centroids, st.centroids_hat, st.centroids_lp, st.sizes,
+                           stream=self.stream)
+        if ev_decode is not None:
+            ev_decode[0].record(self.stream)
+        st.select(self.q)
+        st.decode(self.q, self.K, self.V)
+        if ev_decode is not None:
+            ev_decode[1].record(self.stream)
+
+    def flush_l2(self):
+        self.flush.random_(0, 255)  # a write larger than L2, outside the timed events
+
+
+def time_decode_steps(step: Step, n: int):
+    """Decode steps alone (select + sparse decode), each with L2 flushed first."""
+    times = []
+    for i in range(n):
+        step.flush_l2()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(step.stream)
+        step.st.select(step.q)
+        step.st.decode(step.q, step.K, step.V)
+        b.record(step.stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b) * 1e-3)
+    return times
+
+
+def e2e_measure(w: synth.Workload, dev, stream, steps: int):
+    """End to end through the public calls: pinned host K/V/q -> device, one
+    ckv_cluster + ckv_select + ckv_sparse_decode, outputs -> pinned host."""
+    Kh = torch.empty((w.P, w.L_cap, w.d), dtype=w.torch_dtype, pin_memory=True)
+    Vh = torch.empty_like(Kh, pin_memory=True)
+    Kd, Vd = synth.make_kv(w, device=dev)
+    Kh.copy_(Kd)
+    Vh.copy_(Vd)
+    qh = synth.make_queries(w, device=dev).cpu().pin_memory()
+    st = ClusterRecall(w.P, w.G, w.d, w.torch_dtype, w.L_cap, w.S, w.B, w.C, w.N, w.W, dev,
+                       stream=stream)
+    qd = torch.empty(qh.shape, dtype=qh.dtype, device=dev)
+    out_h = torch.empty((w.P, w.G, w.d), dtype=torch.float32, pin_memory=True)
+    sel_h = torch.empty((w.P, w.B), dtype=torch.int32, pin_memory=True)
+    cnt_h = torch.empty((w.P,), dtype=torch.int32, pin_memory=True)
+    h2d = (Kh.numel() + Vh.numel() + qh.numel()) * Kh.element_size()
+    d2h = out_h.numel() * 4 + sel_h.numel() * 4 + cnt_h.numel() * 4
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(steps + 1):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            qd.copy_(qh, non_blocking=True)
+            st.prefill(Kd, w.L, w.W, w.C, w.T)
+            st.step(qd, Kd, Vd)
+            out_h.copy_(st.out, non_blocking=True)
+            sel_h.copy_(st.sel_idx[:, :w.B], non_blocking=True)
+            cnt_h.copy_(st.sel_cnt, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            if i > 0:  # the first is a warm-up
+                times.append(a.elapsed_time(b) * 1e-3)
+    return statistics.mean(times), h2d, d2h
+
+
+def cpu_baseline(w: synth.Workload, budget_s: float = 20.0):
+    """The oracle (test infrastructure, as it stands) on a bounded sample of the
+    workload: one clustering round (init + assign + update + index) of a few
+    problems, one problem per host thread; keys/s extrapolated to T rounds."""
+    import numpy as np
+    import oracle
+    cores = oracle.threads_default()
+    n_prob = max(1, min(w.P, cores))
+    K, _ = synth.make_kv(w, device="cpu", problems=list(range(n_prob)))
+    Kh = K.float().numpy()
+    tb, te = w.S, w.L - w.W
+    mode = w.dtype
+
+    def one(p):
+        return oracle.kmeans(Kh[p, tb:te], w.C, 1, mode, tok_begin=tb)
+
+    t0 = time.perf_counter()
+    oracle.map_problems(one, list(range(n_prob)), threads=n_prob)
+    dt = time.perf_counter() - t0
+    keys_per_s = n_prob * w.N / (dt * w.T)
+    return {"value": keys_per_s, "unit": "keys/s", "cores": n_prob, "kind": "oracle",
+            "sample": f"{n_prob} of {w.P} problems x 1 of {w.T} k-means rounds "
+                      f"({w.N} keys, C={w.C}, {mode}); keys/s = keys / (round time x {w.T})",
+            "seconds": dt}
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    w = synth.WORKLOADS[args.workload]
+    pk = peaks()
+    with torch.cuda.stream(stream):
+        step = Step(w, dev, stream)
+        torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            step.flush_l2()
+            step.run()
+        torch.cuda.synchronize()
+        ev_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)]
+        ev_assign = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(w.T)] for _ in range(args.steps)]
+        ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            for k in range(args.steps):
+                step.flush_l2()
+                ev_steps[k][0].record(stream)
+                step.run(ev_assign[k], ev_dec[k])
+                ev_steps[k][1].record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        step_s = [a.elapsed_time(b) * 1e-3 for a, b in ev_steps]
+        assign_s = [a.elapsed_time(b) * 1e-3 for row in ev_assign for a, b in row]
+        dec_in_step = [a.elapsed_time(b) * 1e-3 for a, b in ev_dec]
+        total = reduce_max(sum(step_s), world, dev)
+        dec_steps = time_decode_steps(step, max(20, args.steps * 4))
+        err = ckv.ckv_device_error()
+        e2e_s, h2d, d2h = e2e_measure(w, dev, stream, max(2, min(args.steps, 3)))
+        e2e_s = reduce_max(e2e_s, world, dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    keys = w.P * w.N
+    ms_per_step = total / args.steps * 1e3
+    value = world * keys * args.steps / total
+    flops = 2.0 * w.N * w.C * w.d * w.P
+    t_assign = statistics.mean(assign_s)
+    achieved_tf = flops / t_assign / 1e12
+    dec_bytes = decode_bytes(w)
+    t_dec = statistics.median(dec_steps)
+    launches = step.launches_per_step * args.steps
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "keys/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded mixture keys, N(0,1) values; see semantic_cluster_recall_b200/synth.py)",
+        "config": {"workload": w.name, "P": w.P, "L": w.L, "d": w.d, "C": w.C, "T": w.T,
+                   "B": w.B, "sink": w.S, "window": w.W, "N_clustered": w.N, "G": w.G,
+                   "parallelism": f"replicas x{world} (independent problems per GPU)",
+                   "l2": "flushed between timed steps (256 MB write outside the events)",
+                   "step": "init + T x (assign, index, update) + select + sparse decode"},
+        "roofline": {"bound": "tensor", "kernel": "assign (K1)", "achieved": achieved_tf,
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved_tf / pk["bf16_tflops"],
+                     "peak_source": pk["source"] + " bf16 burst",
+                     "traffic": kernel_traffic("assign"),
+                     "flops_per_launch": flops, "us_per_launch": t_assign * 1e6},
+        "decode": {"steps_per_s": 1.0 / t_dec, "us_per_step": t_dec * 1e6,
+                   "us_per_step_in_pipeline": statistics.mean(dec_in_step) * 1e6,
+                   "bytes_per_step": dec_bytes,
+                   "roofline": {"bound": "hbm", "achieved": dec_bytes / t_dec / 1e9,
+                                "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                "frac": dec_bytes / t_dec / 1e9 / pk["hbm_gbs"],
+                                "peak_source": pk["source"] + " copy"},
+                   "l2": "flushed before every decode step"},
+        "e2e": {"value": world * keys / e2e_s, "unit": "keys/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
+        "gpu_launches": launches,
+        "device_error_flags": err,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    line["clocks"] = clk.summary()
+    print(json.dumps(line), flush=True)
+
+
+def decode_bytes(w: synth.Workload) -> float:
+    """Algorithmic bytes of one decode step: every attended K and V row once,
+    the scoring copy of every centroid, q, the output and the selection."""
+    esz = 2 if w.dtype == "bf16" else 4
+    rows = w.S + min(w.B, w.N) + w.W
+    per_problem = (rows * 2 * w.d * esz + w.C * w.d * esz + w.G * w.d * esz + w.G * w.d * 4
+                   + min(w.B, w.N) * 4 * 2 + (w.C + 1) * 4)
+    return float(w.P * per_problem)
+
+
+# ---------------------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------------------
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        cpu_baseline(w)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = cpu_baseline(w)
+        vals.append(r["value"])
+        secs.append(r["seconds"])
+    v = statistics.mean(vals)
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": v,
+        "unit": "keys/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": statistics.mean(secs) * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded mixture keys)",
+        "config": {"workload": w.name, "P": w.P, "L": w.L, "d": w.d, "C": w.C, "T": w.T,
+                   "B": w.B, "sink": w.S, "window": w.W, "N_clustered": w.N},
+        "cpu_baseline": {"value": v, "unit": "keys/s", "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

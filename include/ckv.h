@@ -1,0 +1,232 @@
+/*
+ * ckv.h -- C ABI of libckv.so: B200 (sm_100a) kernels for ClusterKV-style
+ * semantic cluster recall of the KV cache.
+ *
+ * Method: "ClusterKV: Manipulating LLM KV Cache in Semantic Space for
+ * Recallable Compression" (Liu, Li, Zhao, Zhang, Guo; arXiv 2412.03213v2),
+ * as summarised section by section on its paperlayer.ai page. After prefill,
+ * each KV head's keys are grouped by cosine k-means ("III.B Clustering in the
+ * Semantic Space"); the centroids, cluster sizes, their prefix sums and the
+ * token indices sorted by cluster are kept ("IV.C Selection and Indexing");
+ * at each decode step the query ranks the clusters by attention weight and
+ * whole clusters are recalled until a token budget is met, the last one
+ * trimmed ("IV.C Selection and Indexing", "III.C Selection at the Granularity
+ * of Semantic Clusters"); attention then runs over the recalled tokens plus
+ * the attention-sink and recent tokens ("II.A LLM Inference and KV Cache").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - A "problem" is one (layer, batch, KV head). P problems are processed per
+ *   call; problem p's data sits at base + p * stride.
+ * - d (head dimension) must be 128.
+ * - dtype: CKV_BF16 (bf16 storage, fp32 accumulation; the clustering
+ *   similarity runs on tcgen05 tensor cores) or CKV_F32 (fp32 storage and
+ *   arithmetic on CUDA cores).
+ * - All pointers are device memory owned by the caller. The library allocates
+ *   nothing, keeps no state between calls other than a device error word (see
+ *   ckv_device_error) and cached per-device attributes, and never
+ *   synchronises except in ckv_device_error.
+ * - Every call is asynchronous and ordered on `stream` (a cudaStream_t passed
+ *   as void*; NULL is the legacy default stream).
+ * - Arguments are validated on the host before anything is launched; a bad
+ *   argument returns CKV_ERR_INVALID and launches nothing. A launch failure
+ *   returns CKV_ERR_CUDA. ckv_last_error() gives a one-line reason for the
+ *   calling thread's last failure.
+ * - Device-side checks: an out-of-range label, perm entry, selected index or
+ *   tail position is skipped (never dereferenced) and sets a bit in the
+ *   device error word instead of faulting.
+ *
+ * Region layout inside each problem
+ * ---------------------------------
+ *   positions [0, sink)                attention sinks, always attended
+ *   positions [tok_begin, tok_end)     clustered tokens (prefill: [sink, L-W))
+ *   positions [tail_begin, tail_end)   recent tokens, attended densely
+ * Cluster metadata arrays are sized by capacities so that clusters of
+ * generated tokens can be appended later ("III.B": every so many decode steps
+ * the generated tokens alone are clustered into a few new centroids):
+ *   centroids      float [P][C_cap][d]   mu: the mean of the raw member keys
+ *   centroids_hat  dtype [P][C_cap][d]   mu / ||mu|| rounded to dtype: the
+ *                                        copy the assignment step uses
+ *   centroids_lp   dtype [P][C_cap][d]   mu rounded to dtype: the copy the
+ *                                        decode-time scoring uses
+ *   sizes          int32 [P][C_cap]      members per cluster
+ *   offsets        int32 [P][C_cap + 1]  start of cluster c in perm (absolute
+ *                                        slot); cluster c owns slots
+ *                                        [offsets[c], offsets[c+1])
+ *   labels         int32 [P][perm_cap]   slot perm_base + i holds the cluster
+ *                                        id (cluster_base + local id) of token
+ *                                        tok_begin + i
+ *   perm           int32 [P][perm_cap]   token positions grouped by cluster,
+ *                                        ascending within each cluster
+ * A clustering call writes clusters [cluster_base, cluster_base + C) and perm
+ * slots [perm_base, perm_base + tok_end - tok_begin); the prefill call uses
+ * (0, 0) and an appended call continues where the previous one ended.
+ */
+#ifndef CKV_H
+#define CKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CKV_OK = 0,
+    CKV_ERR_INVALID = 1,     /* bad argument; nothing was launched */
+    CKV_ERR_CUDA = 2,        /* a CUDA launch or runtime call failed */
+    CKV_ERR_TIMEOUT = 3,     /* a bounded device wait gave up */
+    CKV_ERR_UNSUPPORTED = 4  /* valid but not implemented (dtype/shape) */
+} ckv_status;
+
+typedef enum { CKV_F32 = 0, CKV_BF16 = 1 } ckv_dtype;
+
+/* Device error bits (see ckv_device_error). */
+#define CKV_DEVERR_LABEL 0x1u   /* a label outside [cluster_base, cluster_base+C) */
+#define CKV_DEVERR_PERM 0x2u    /* a perm entry outside [tok_begin, tok_end) */
+#define CKV_DEVERR_INDEX 0x4u   /* a selected / tail position outside the K/V rows */
+#define CKV_DEVERR_OFFSETS 0x8u /* offsets not monotone or outside [0, perm_cap] */
+
+/* Largest supported number of clusters per problem (C_cap). */
+#define CKV_MAX_CLUSTERS 4096
+
+const char *ckv_status_string(int status);
+/* One-line reason for the calling thread's last non-OK status ("" if none). */
+const char *ckv_last_error(void);
+int ckv_version(void);
+
+/* Read (and optionally clear) the device error word of the current device.
+ * Synchronises `stream`. *flags receives the CKV_DEVERR_* bits. */
+ckv_status ckv_device_error(unsigned int *flags, int clear, void *stream);
+
+/* ---- clustering --------------------------------------------------------- */
+
+/* Workspace for ckv_cluster / ckv_index: per-chunk cluster histograms.
+ * n_tok = tok_end - tok_begin. */
+size_t ckv_index_workspace_bytes(int P, int n_tok, int C);
+size_t ckv_cluster_workspace_bytes(int P, int n_tok, int C);
+
+/* Cosine k-means over the keys of [tok_begin, tok_end) of every problem
+ * ("III.B Clustering in the Semantic Space": assign each key to the centroid
+ * of highest cosine similarity, move each centroid to the mean of its keys).
+ * Seeding: centroid c starts at the key of position tok_begin + c * floor(n/C)
+ * (the paper does not say how it seeds). Exactly `iters` rounds of (assign,
+ * update) run; there is no early exit. On return: labels are the last round's
+ * assignment, centroids the means of exactly those clusters (a cluster that
+ * ended empty keeps its previous centroid), and sizes/offsets/perm the index
+ * of those labels ("IV.C Selection and Indexing").
+ *   keys            dtype, problem p's row t at keys + p*problem_stride + t*d
+ *   problem_stride  elements between problems (>= tok_end * d)
+ *   C, iters        1 <= C <= n_tok, C <= C_cap - cluster_base; iters >= 1
+ *   workspace       >= ckv_cluster_workspace_bytes(P, n_tok, C) bytes, any
+ *                   contents, 256-byte aligned
+ * Errors: CKV_ERR_INVALID for null pointers, d != 128, C < 1, n_tok < C,
+ * iters < 1, capacities exceeded, a small or misaligned workspace. */
+ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                       int tok_begin, int tok_end, int C, int iters, int cluster_base,
+                       int perm_base, int C_cap, int perm_cap, float *centroids,
+                       void *centroids_hat, void *centroids_lp, int32_t *labels,
+                       int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
+                       size_t ws_bytes, void *stream);
+
+/* Stage: strided seeding only (mu, mu-hat and the scoring copy of clusters
+ * [cluster_base, cluster_base + C)). Arguments as in ckv_cluster. */
+ckv_status ckv_init_centroids(const void *keys, ckv_dtype dt, int P, int64_t problem_stride,
+                              int d, int tok_begin, int tok_end, int C, int cluster_base,
+                              int C_cap, float *centroids, void *centroids_hat,
+                              void *centroids_lp, void *stream);
+
+/* Stage: assignment. labels[p][perm_base + i] = cluster_base + argmax_c
+ * (k_i . centroids_hat[c]) over c in [0, C), ties to the lowest c. For bf16
+ * this is a bf16 x bf16 -> fp32 tensor-core contraction with the argmax fused
+ * into its epilogue; for fp32 an FFMA contraction. */
+ckv_status ckv_assign(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                      int tok_begin, int tok_end, const void *centroids_hat, int C,
+                      int cluster_base, int C_cap, int32_t *labels, int perm_base, int perm_cap,
+                      void *stream);
+
+/* Stage: cluster index of the labels of slots [perm_base, perm_base + n_tok):
+ * offsets[cluster_base + c] for c in [0, C] (the last one is
+ * perm_base + n_tok) and perm, a stable bucket sort (ascending position within
+ * each cluster). Labels must lie in [cluster_base, cluster_base + C). */
+ckv_status ckv_index(const int32_t *labels, int P, int tok_begin, int tok_end, int C,
+                     int cluster_base, int C_cap, int perm_base, int perm_cap,
+                     int32_t *offsets, int32_t *perm, void *workspace, size_t ws_bytes,
+                     void *stream);
+
+/* Stage: centroid update from an index: for each cluster c in
+ * [cluster_base, cluster_base + C), mu_c = mean of the keys at
+ * perm[offsets[c] .. offsets[c+1]) (summed in fp32 in perm order), sizes[c] =
+ * its member count, centroids_hat = mu/||mu|| and centroids_lp = mu, both
+ * rounded to dtype. A cluster with no members or a zero mean keeps its
+ * previous centroids. tok_begin/tok_end bound the valid perm entries. */
+ckv_status ckv_update(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                      int tok_begin, int tok_end, int C, int cluster_base, int C_cap,
+                      const int32_t *offsets, const int32_t *perm, int perm_cap,
+                      float *centroids, void *centroids_hat, void *centroids_lp,
+                      int32_t *sizes, void *stream);
+
+/* ---- decode-time selection ---------------------------------------------- */
+
+size_t ckv_select_workspace_bytes(int P, int C_cap);
+
+/* Cluster-granularity recall ("IV.C Selection and Indexing"). For problem p
+ * with n_clusters[p] clusters:
+ *   score s_c = sum over the G query heads of q_g . centroids_lp[c], computed
+ *     in fp32 in a fixed order (channels split in 32 groups of 4, each summed
+ *     with fmaf from 0 in channel order, the groups combined by an xor
+ *     butterfly over 16, 8, 4, 2, 1, then heads added in order). The softmax
+ *     is monotone, so ranking by this logit ranks by attention weight.
+ *   rank: clusters by descending score, ties to the lower cluster id;
+ *   fill: clusters are taken whole while they fit in the budget; the first
+ *     that does not fit contributes its first (lowest-position) tokens up to
+ *     the budget and the walk stops.
+ * Output: sel_idx[p][0 .. sel_cnt[p]) token positions in rank order, then perm
+ * order; sel_cnt[p] = min(budget, total clustered tokens).
+ *   q             dtype [P][G][d]
+ *   n_clusters    int32 [P] (device), each in [0, C_cap]
+ *   budget        >= 0; sel_idx has row stride `budget`
+ *   G             1..8 */
+ckv_status ckv_select(const void *q, ckv_dtype dt, int P, int G, int d,
+                      const void *centroids_lp, const int32_t *n_clusters, int C_cap,
+                      const int32_t *offsets, const int32_t *perm, int perm_cap, int budget,
+                      int32_t *sel_idx, int32_t *sel_cnt, void *workspace, size_t ws_bytes,
+                      void *stream);
+
+/* ---- sparse decode attention -------------------------------------------- */
+
+/* max_rows bounds sink + budget + (tail_end - tail_begin) over all problems. */
+size_t ckv_decode_workspace_bytes(int P, int G, int d, int max_rows);
+
+/* out[p][g] = sum_{j in A} softmax_j(scale * q_g . k_j) v_j with
+ * A = [0, sink) + sel_idx[p][0..sel_cnt[p]) + [tail_begin[p], tail_end[p])
+ * ("II.A LLM Inference and KV Cache"; the attended set is the paper's
+ * selected tokens plus sinks and recent tokens). Split-K over A with an
+ * fp32 online softmax; partial results are merged by a second kernel.
+ *   q            dtype [P][G][d];  K, V dtype, row t of problem p at
+ *                base + p*kv_problem_stride + t*d; kv_rows rows per problem
+ *   tail_begin/tail_end  int32 [P] (device)
+ *   max_tail     upper bound of tail_end - tail_begin (grid sizing)
+ *   out          float [P][G][d]
+ *   workspace    >= ckv_decode_workspace_bytes(P, G, d, sink + budget +
+ *                max_tail) bytes, 256-byte aligned */
+ckv_status ckv_sparse_decode(const void *q, const void *K, const void *V, ckv_dtype dt, int P,
+                             int G, int d, int64_t kv_problem_stride, int kv_rows, int sink,
+                             const int32_t *tail_begin, const int32_t *tail_end, int max_tail,
+                             const int32_t *sel_idx, const int32_t *sel_cnt, int budget,
+                             float scale, float *out, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/* Append one generated token per problem: K/V row tail_end[p] <- new_k[p] /
+ * new_v[p] (dtype [P][d]); then tail_end[p] += 1. A full cache (tail_end[p]
+ * >= kv_rows) writes nothing and sets CKV_DEVERR_INDEX. */
+ckv_status ckv_append(void *K, void *V, ckv_dtype dt, int P, int d, int64_t kv_problem_stride,
+                      int kv_rows, const void *new_k, const void *new_v, int32_t *tail_end,
+                      void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKV_H */

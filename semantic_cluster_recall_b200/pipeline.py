@@ -1,0 +1,119 @@
+"""Device-memory holder and call sequencing for the three C-ABI stages.
+
+ClusterRecall owns the caller-side buffers that libckv needs (centroids,
+cluster index, selections, workspaces) as torch CUDA tensors and sequences the
+entry points of ckv.py for a batch of P independent (layer, batch, KV-head)
+problems:
+
+* prefill(K): cosine k-means of positions [S, L - W) of every problem
+  ("III.B Clustering in the Semantic Space" of "ClusterKV: Manipulating LLM KV
+  Cache in Semantic Space for Recallable Compression", arXiv 2412.03213v2);
+* select(q): cluster-granularity recall under the token budget ("IV.C
+  Selection and Indexing");
+* decode(q): attention over sinks + recalled + recent tokens;
+* append(k, v) / incremental(): one generated token per step, and clustering
+  of the oldest generated tokens into a few new clusters once the recent tail
+  reaches its capacity ("III.B": generated tokens are clustered on their own
+  into four new centroids every so many steps).
+
+Nothing here computes: every step is one of libckv's kernels.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import ckv
+
+
+class ClusterRecall:
+    def __init__(self, P: int, G: int, d: int, dtype: torch.dtype, kv_rows: int, S: int,
+                 budget: int, C_cap: int, perm_cap: int, max_tail: int, device,
+                 stream: Optional[torch.cuda.Stream] = None):
+        if d != 128:
+            raise ValueError("d must be 128")
+        self.P, self.G, self.d, self.dtype = P, G, d, dtype
+        self.kv_rows, self.S, self.B = kv_rows, S, budget
+        self.C_cap, self.perm_cap, self.max_tail = C_cap, perm_cap, max_tail
+        self.device = torch.device(device)
+        self.stream = stream
+        dev = self.device
+        i32 = torch.int32
+        self.centroids = torch.zeros((P, C_cap, d), dtype=torch.float32, device=dev)
+        self.centroids_hat = torch.zeros((P, C_cap, d), dtype=dtype, device=dev)
+        self.centroids_lp = torch.zeros((P, C_cap, d), dtype=dtype, device=dev)
+        self.sizes = torch.zeros((P, C_cap), dtype=i32, device=dev)
+        self.offsets = torch.zeros((P, C_cap + 1), dtype=i32, device=dev)
+        self.labels = torch.zeros((P, perm_cap), dtype=i32, device=dev)
+        self.perm = torch.zeros((P, perm_cap), dtype=i32, device=dev)
+        self.n_clusters = torch.zeros((P,), dtype=i32, device=dev)
+        self.tail_begin = torch.zeros((P,), dtype=i32, device=dev)
+        self.tail_end = torch.zeros((P,), dtype=i32, device=dev)
+        self.sel_idx = torch.zeros((P, max(budget, 1)), dtype=i32, device=dev)
+        self.sel_cnt = torch.zeros((P,), dtype=i32, device=dev)
+        self.out = torch.zeros((P, G, d), dtype=torch.float32, device=dev)
+        self.ws_select = ckv.workspace(ckv.ckv_select_workspace_bytes(P, C_cap), dev)
+        self.ws_decode = ckv.workspace(
+            ckv.ckv_decode_workspace_bytes(P, G, d, S + budget + max_tail), dev)
+        self.ws_cluster: Optional[torch.Tensor] = None
+        # host-side bookkeeping of the clustered region (same for all problems)
+        self.n_clustered = 0      # perm slots used
+        self.C_used = 0           # clusters used
+        self.tail_lo = 0          # host copy of tail_begin (uniform over problems)
+        self.scale = 1.0 / math.sqrt(d)
+
+    def _ws_cluster(self, n_tok: int, C: int) -> torch.Tensor:
+        need = ckv.ckv_cluster_workspace_bytes(self.P, n_tok, C)
+        if self.ws_cluster is None or self.ws_cluster.numel() < need:
+            self.ws_cluster = ckv.workspace(need, self.device)
+        return self.ws_cluster
+
+    def prefill(self, K: torch.Tensor, L: int, W: int, C: int, iters: int):
+        """Cluster positions [S, L - W); the last W prompt tokens start the tail."""
+        tb, te = self.S, L - W
+        ws = self._ws_cluster(te - tb, C)
+        ckv.ckv_cluster(K, K.stride(0), tb, te, C, iters, 0, 0, self.C_cap, self.perm_cap,
+                        self.centroids, self.centroids_hat, self.centroids_lp, self.labels,
+                        self.sizes, self.offsets, self.perm, ws, P=self.P, d=self.d,
+                        stream=self.stream)
+        self.n_clustered, self.C_used, self.tail_lo = te - tb, C, te
+        self.n_clusters.fill_(C)
+        self.tail_begin.fill_(te)
+        self.tail_end.fill_(L)
+
+    def incremental(self, K: torch.Tensor, n_tok: int, C: int, iters: int):
+        """Cluster the oldest n_tok tail tokens into C new clusters appended to
+        the metadata; the tail then starts after them."""
+        tb, te = self.tail_lo, self.tail_lo + n_tok
+        ws = self._ws_cluster(n_tok, C)
+        ckv.ckv_cluster(K, K.stride(0), tb, te, C, iters, self.C_used, self.n_clustered,
+                        self.C_cap, self.perm_cap, self.centroids, self.centroids_hat,
+                        self.centroids_lp, self.labels, self.sizes, self.offsets, self.perm, ws,
+                        P=self.P, d=self.d, stream=self.stream)
+        self.n_clustered += n_tok
+        self.C_used += C
+        self.tail_lo = te
+        self.n_clusters.fill_(self.C_used)
+        self.tail_begin.fill_(te)
+
+    def select(self, q: torch.Tensor):
+        ckv.ckv_select(q, self.centroids_lp, self.n_clusters, self.C_cap, self.offsets, self.perm,
+                       self.perm_cap, self.B, self.sel_idx, self.sel_cnt, self.ws_select,
+                       P=self.P, G=self.G, d=self.d, stream=self.stream)
+
+    def decode(self, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor) -> torch.Tensor:
+        ckv.ckv_sparse_decode(q, K, V, K.stride(0), self.kv_rows, self.S, self.tail_begin,
+                              self.tail_end, self.max_tail, self.sel_idx, self.sel_cnt, self.B,
+                              self.scale, self.out, self.ws_decode, P=self.P, G=self.G,
+                              d=self.d, stream=self.stream)
+        return self.out
+
+    def step(self, q, K, V) -> torch.Tensor:
+        self.select(q)
+        return self.decode(q, K, V)
+
+    def append(self, K, V, new_k, new_v):
+        ckv.ckv_append(K, V, K.stride(0), self.kv_rows, new_k, new_v, self.tail_end, P=self.P,
+                       d=self.d, stream=self.stream)

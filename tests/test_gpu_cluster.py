@@ -1,0 +1,95 @@
+"""End-to-end parity of ckv_cluster (all rounds in one call) with the oracle.
+
+k-means is an iteration: one label that flips at a near-tie moves a centroid
+and the two runs then follow different trajectories. So the GPU result after
+t rounds (t = 1..T, each a fresh deterministic call) is compared with the
+oracle's round-t labels; at the first round where they differ, every differing
+token must be an exempt near-tie of the oracle (top-2 cosine gap < 1e-4 under
+the oracle's centroids of that round), and up to that round the centroids
+agree within 1e-3 relative L2. On well-separated data (no near-ties) the whole
+run, including the index and the centroids, must agree.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semantic_cluster_recall_b200 import ckv, synth
+from semantic_cluster_recall_b200.pipeline import ClusterRecall
+
+from helpers import (CENT_REL_L2, GAP_EXEMPT, OUT_MAX_ABS, centroid_rel_err, f32np,
+                     oracle_kmeans_all, small_workload)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_gpu(K, w, iters, dev):
+    st = ClusterRecall(w.P, w.G, 128, K.dtype, K.shape[1], w.S, w.B, w.C + 4, w.N + 8, w.W, dev)
+    st.prefill(K, w.L, w.W, w.C, iters)
+    torch.cuda.synchronize()
+    return st
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_cluster_first_divergence_is_a_near_tie(cuda_device, dtype):
+    w = small_workload(dtype, P=3, L=4000, C=60, T=6)
+    K, _ = synth.make_kv(w)
+    Kh = f32np(K)
+    Kd = K.to(cuda_device)
+    n = w.N
+    live = set(range(w.P))  # problems whose trajectories still agree
+    for t in range(1, w.T + 1):
+        st = _run_gpu(Kd, w.replace(T=t), t, cuda_device)
+        refs = oracle_kmeans_all(Kh, w.replace(T=t), history=True)
+        for p in sorted(live):
+            r = refs[p]
+            lab = st.labels[p, :n].cpu().numpy()
+            if not np.array_equal(lab, r["labels"]):
+                gap = r["gap_hist"][t - 1]
+                bad = (lab != r["labels"]) & (gap >= GAP_EXEMPT)
+                assert not bad.any(), f"p={p} round {t}: {bad.sum()} non-tie label differences"
+                live.discard(p)
+                continue
+            # same labels up to round t: index bit-exact, centroids within tolerance
+            assert np.array_equal(st.offsets[p, :w.C + 1].cpu().numpy(), r["offsets"])
+            assert np.array_equal(st.perm[p, :n].cpu().numpy(), r["perm"])
+            assert np.array_equal(st.sizes[p, :w.C].cpu().numpy(), r["sizes"])
+            err = centroid_rel_err(f32np(st.centroids[p, :w.C]), r["mu"])
+            assert err.max() <= CENT_REL_L2, (p, t, err.max())
+    assert ckv.ckv_device_error() == 0
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_whole_path_on_well_separated_mixture(cuda_device, G):
+    # well separated (small noise) and a peaked query: no near-ties, so the GPU
+    # and the oracle follow the same trajectory and every output can be compared
+    w = small_workload(torch.bfloat16, P=4, G=G, L=6000, C=48, T=5, B=700, M=48,
+                       sigma=0.3 / np.sqrt(128), q_scale=8.0)
+    K, V = synth.make_kv(w)
+    q = synth.make_queries(w)
+    Kh, Vh, qh = f32np(K), f32np(V), f32np(q)
+    dev = cuda_device
+    Kd, Vd, qd = K.to(dev), V.to(dev), q.to(dev)
+    st = _run_gpu(Kd, w, w.T, dev)
+    out = st.step(qd, Kd, Vd)
+    torch.cuda.synchronize()
+    refs = oracle_kmeans_all(Kh, w, history=True)
+    n = w.N
+    for p in range(w.P):
+        r = refs[p]
+        assert r["gap_hist"].min() >= GAP_EXEMPT  # the premise: no near-ties
+        assert np.array_equal(st.labels[p, :n].cpu().numpy(), r["labels"])
+        assert np.array_equal(st.offsets[p, :w.C + 1].cpu().numpy(), r["offsets"])
+        assert np.array_equal(st.perm[p, :n].cpu().numpy(), r["perm"])
+        assert centroid_rel_err(f32np(st.centroids[p, :w.C]), r["mu"]).max() <= CENT_REL_L2
+        # selection from the GPU's own centroids and the oracle's: compared
+        # through the oracle's scoring of the GPU's scoring copy
+        lp_gpu = f32np(st.centroids_lp[p, :w.C])
+        s = oracle.score(qh[p], lp_gpu)
+        sel, cnt = oracle.select(s, r["offsets"], r["perm"], w.B)
+        assert st.sel_cnt[p].item() == cnt
+        assert np.array_equal(st.sel_idx[p, :cnt].cpu().numpy(), sel)
+        rows = oracle.attended_rows(w.S, sel, w.L - w.W, w.L)
+        ref_out = oracle.attend(qh[p], Kh[p], Vh[p], rows, 1 / np.sqrt(128))
+        assert np.abs(out[p].cpu().numpy() - ref_out).max() <= OUT_MAX_ABS
+    assert ckv.ckv_device_error() == 0

@@ -1,0 +1,269 @@
+"""Stage-by-stage (teacher-forced) parity of the CUDA path with the CPU oracle.
+
+Every stage gets its inputs from the oracle (or the seeded generator) and its
+output is compared with the oracle's output for the same inputs:
+  init    exact for fp32, bf16 unit copy within one bf16 ulp
+  assign  labels equal except where the oracle's top-2 cosine gap < 1e-4
+  index   offsets and perm bit-exact
+  update  sizes exact, centroids within 1e-3 relative L2
+  select  sel_idx / sel_cnt bit-exact (scores in the same fp32 order)
+  decode  within 2e-3 max-abs of the oracle's double attention
+All calls go through the C ABI (libckv.so) via the ctypes binding.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semantic_cluster_recall_b200 import ckv, synth
+
+from helpers import (CENT_REL_L2, GAP_EXEMPT, OUT_MAX_ABS, centroid_rel_err, f32np, mode_of,
+                     oracle_kmeans_all, small_workload, to_dev, labels_match_except_near_ties)
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = [torch.bfloat16, torch.float32]
+
+
+def _kv(w, dev):
+    K, V = synth.make_kv(w, device="cpu")
+    return K.to(dev), V.to(dev), f32np(K), f32np(V)
+
+
+# ---- init ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_init_matches_oracle(cuda_device, dtype):
+    w = small_workload(dtype, P=3, L=2500, C=77)
+    K, V, Kh, _ = _kv(w, cuda_device)
+    P, C_cap = w.P, w.C + 5
+    cent = torch.zeros((P, C_cap, 128), device=cuda_device)
+    hat = torch.zeros((P, C_cap, 128), dtype=dtype, device=cuda_device)
+    lp = torch.zeros_like(hat)
+    tb, te = w.S, w.L - w.W
+    ckv.ckv_init_centroids(K, K.stride(0), tb, te, w.C, 2, C_cap, cent, hat, lp)
+    torch.cuda.synchronize()
+    for p in range(P):
+        mu, muhat = oracle.init(Kh[p, tb:te], w.C, mode_of(dtype))
+        np.testing.assert_array_equal(f32np(cent[p, 2:2 + w.C]), mu.astype(np.float32))
+        np.testing.assert_array_equal(f32np(lp[p, 2:2 + w.C]), mu.astype(np.float32))
+        got = f32np(hat[p, 2:2 + w.C]).astype(np.float64)
+        # one storage ulp: the GPU normalises in fp32, the oracle in double
+        ulp = 2.0 ** -7 if dtype == torch.bfloat16 else 1e-6
+        np.testing.assert_allclose(got, muhat, rtol=ulp, atol=1e-30)
+
+
+# ---- assign ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("C,L", [(50, 3000), (400, 4200), (7, 700), (1, 300), (260, 2200)])
+def test_assign_matches_oracle_except_near_ties(cuda_device, dtype, C, L):
+    w = small_workload(dtype, P=2, L=L, C=C, M=max(C, 8))
+    K, V, Kh, _ = _kv(w, cuda_device)
+    tb, te = w.S, w.L - w.W
+    n = te - tb
+    P, C_cap, perm_cap = w.P, C + 3, n + 11
+    mode = mode_of(dtype)
+    # teacher-forced centroids: the oracle's unit copy after one round
+    hats = []
+    for p in range(P):
+        r = oracle.kmeans(Kh[p, tb:te], C, 1, mode)
+        hats.append(r["muhat"])
+    hat_np = np.zeros((P, C_cap, 128), np.float32)
+    for p in range(P):
+        hat_np[p, 3:3 + C] = hats[p]
+    hat = to_dev(hat_np, dtype, cuda_device)
+    labels = torch.full((P, perm_cap), -7, dtype=torch.int32, device=cuda_device)
+    ckv.ckv_assign(K, K.stride(0), tb, te, hat, C, 3, C_cap, labels, 5, perm_cap)
+    torch.cuda.synchronize()
+    lab = labels.cpu().numpy()
+    for p in range(P):
+        ref, gap = oracle.assign(Kh[p, tb:te], hats[p])
+        got = lab[p, 5:5 + n] - 3
+        ndiff, nbad, _ = labels_match_except_near_ties(got, ref, gap)
+        assert nbad == 0, f"problem {p}: {nbad} label mismatches outside near-ties ({ndiff} total)"
+        assert np.all(lab[p, :5] == -7) and np.all(lab[p, 5 + n:] == -7)
+
+
+# ---- index -----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,C,skew", [(5000, 37, 0.0), (2048, 400, 1.1), (33, 64, 0.0),
+                                      (1, 1, 0.0), (20000, 1600, 0.7), (4097, 3, 0.0)])
+def test_index_bit_exact(cuda_device, n, C, skew):
+    P, tb, cb, pb = 3, 40, 6, 9
+    C_cap, perm_cap = cb + C + 2, pb + n + 5
+    lab_local = synth.random_labels(P, n, C, seed=n * 7 + C, skew=skew).numpy()
+    labels_np = np.full((P, perm_cap), -1, np.int32)
+    labels_np[:, pb:pb + n] = lab_local + cb
+    labels = torch.from_numpy(labels_np).to(cuda_device)
+    offsets = torch.full((P, C_cap + 1), -5, dtype=torch.int32, device=cuda_device)
+    perm = torch.full((P, perm_cap), -5, dtype=torch.int32, device=cuda_device)
+    ws = ckv.workspace(ckv.ckv_index_workspace_bytes(P, n, C), cuda_device)
+    ckv.ckv_index(labels, P, tb, tb + n, C, cb, C_cap, pb, perm_cap, offsets, perm, ws)
+    torch.cuda.synchronize()
+    off, pm = offsets.cpu().numpy(), perm.cpu().numpy()
+    for p in range(P):
+        ro, rp = oracle.index(lab_local[p], C, tb, pb)
+        assert np.array_equal(off[p, cb:cb + C + 1], ro)
+        assert np.array_equal(pm[p, pb:pb + n], rp)
+        assert np.all(off[p, :cb] == -5) and np.all(off[p, cb + C + 1:] == -5)
+        assert np.all(pm[p, :pb] == -5) and np.all(pm[p, pb + n:] == -5)
+    assert ckv.ckv_device_error() == 0
+
+
+# ---- update ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("C,skew", [(50, 0.0), (400, 1.2), (3, 0.0)])
+def test_update_matches_oracle(cuda_device, dtype, C, skew):
+    w = small_workload(dtype, P=2, L=3000, C=C)
+    K, V, Kh, _ = _kv(w, cuda_device)
+    tb, te = w.S, w.L - w.W
+    n = te - tb
+    P, cb, C_cap, perm_cap = w.P, 2, C + 4, n + 3
+    mode = mode_of(dtype)
+    lab = synth.random_labels(P, n, C, seed=C + 99, skew=skew).numpy()
+    mu0 = np.random.default_rng(1).standard_normal((P, C, 128)).astype(np.float32)
+    cent_np = np.zeros((P, C_cap, 128), np.float32)
+    cent_np[:, cb:cb + C] = mu0
+    hat0 = oracle.round_to(mu0, mode).astype(np.float32)
+    hat_np = np.zeros((P, C_cap, 128), np.float32)
+    hat_np[:, cb:cb + C] = hat0
+    cent = torch.from_numpy(cent_np).to(cuda_device)
+    hat = to_dev(hat_np, dtype, cuda_device)
+    lp = hat.clone()
+    sizes = torch.full((P, C_cap), -3, dtype=torch.int32, device=cuda_device)
+    off_np = np.zeros((P, C_cap + 1), np.int32)
+    perm_np = np.zeros((P, perm_cap), np.int32)
+    refs = []
+    for p in range(P):
+        o, pm = oracle.index(lab[p], C, tb, 0)
+        off_np[p, cb:cb + C + 1] = o
+        perm_np[p, :n] = pm
+        refs.append(oracle.update(Kh[p, tb:te], lab[p], mu0[p], hat0[p], mode))
+    ckv.ckv_update(K, K.stride(0), tb, te, C, cb, C_cap, torch.from_numpy(off_np).to(cuda_device),
+                   torch.from_numpy(perm_np).to(cuda_device), perm_cap, cent, hat, lp, sizes)
+    torch.cuda.synchronize()
+    for p in range(P):
+        mu_r, hat_r, sz_r = refs[p]
+        assert np.array_equal(sizes[p, cb:cb + C].cpu().numpy(), sz_r)
+        err = centroid_rel_err(f32np(cent[p, cb:cb + C]), mu_r)
+        assert err.max() <= CENT_REL_L2, err.max()
+        # one storage ulp (bf16), or the fp32 summation error (f32)
+        ulp = 2.0 ** -7 if dtype == torch.bfloat16 else 1e-5
+        np.testing.assert_allclose(f32np(hat[p, cb:cb + C]), hat_r, rtol=ulp, atol=1e-6)
+        lp_ref = oracle.round_to(mu_r, mode)
+        np.testing.assert_allclose(f32np(lp[p, cb:cb + C]), lp_ref, rtol=ulp, atol=1e-6)
+        empty = sz_r == 0
+        if empty.any():  # empty clusters keep their previous centroid bit for bit
+            assert np.array_equal(f32np(cent[p, cb:cb + C])[empty], mu0[p][empty])
+    assert ckv.ckv_device_error() == 0
+
+
+# ---- select ----------------------------------------------------------------------------
+
+def _select_case(cuda_device, dtype, P, G, C, n, budget, seed, ties=False, n_clusters=None):
+    rng = np.random.default_rng(seed)
+    mode = mode_of(dtype)
+    tb, pb = 16, 3
+    C_cap, perm_cap = C + 5, pb + n + 2
+    lab = synth.random_labels(P, n, C, seed=seed, skew=0.8).numpy()
+    mu = rng.standard_normal((P, C, 128))
+    if ties:  # duplicate centroids -> exactly equal scores, resolved by cluster id
+        mu[:, 1::3] = mu[:, 0:-1:3][:, :mu[:, 1::3].shape[1]]
+    mu_lp = oracle.round_to(mu, mode).astype(np.float32)
+    q = oracle.round_to(rng.standard_normal((P, G, 128)), mode).astype(np.float32)
+    ncl = np.full(P, C, np.int32) if n_clusters is None else np.asarray(n_clusters, np.int32)
+    lp_np = np.zeros((P, C_cap, 128), np.float32)
+    lp_np[:, :C] = mu_lp
+    off_np = np.zeros((P, C_cap + 1), np.int32)
+    perm_np = np.full((P, perm_cap), -1, np.int32)
+    refs = []
+    for p in range(P):
+        o, pm = oracle.index(lab[p], C, tb, pb)
+        off_np[p, :C + 1] = o
+        perm_np[p, pb:pb + n] = pm
+        s = oracle.score(q[p], mu_lp[p][:ncl[p]])
+        refs.append(oracle.select(s, o[:ncl[p] + 1], pm, budget, perm_base=pb))
+    dev = cuda_device
+    sel = torch.full((P, max(budget, 1)), -9, dtype=torch.int32, device=dev)
+    cnt = torch.full((P,), -9, dtype=torch.int32, device=dev)
+    ws = ckv.workspace(ckv.ckv_select_workspace_bytes(P, C_cap), dev)
+    ckv.ckv_select(to_dev(q, dtype, dev), to_dev(lp_np, dtype, dev),
+                   torch.from_numpy(ncl).to(dev), C_cap, torch.from_numpy(off_np).to(dev),
+                   torch.from_numpy(perm_np).to(dev), perm_cap, budget, sel, cnt, ws)
+    torch.cuda.synchronize()
+    sel_h, cnt_h = sel.cpu().numpy(), cnt.cpu().numpy()
+    for p in range(P):
+        r_sel, r_cnt = refs[p]
+        assert cnt_h[p] == r_cnt
+        assert np.array_equal(sel_h[p, :r_cnt], r_sel), f"problem {p}"
+    assert ckv.ckv_device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("G", [1, 4])
+@pytest.mark.parametrize("budget", [0, 1, 256, 1024, 5000])
+def test_select_bit_exact(cuda_device, dtype, G, budget):
+    _select_case(cuda_device, dtype, P=4, G=G, C=400, n=4000, budget=budget, seed=budget + G)
+
+
+def test_select_ties_large_C_and_partial_cluster_counts(cuda_device):
+    _select_case(cuda_device, torch.bfloat16, P=3, G=2, C=1604, n=20000, budget=2048, seed=5,
+                 ties=True, n_clusters=[1604, 1600, 17])
+
+
+# ---- decode ----------------------------------------------------------------------------
+
+def _decode_case(cuda_device, dtype, P, G, L, S, sel_counts, tails, budget, q_scale=1.0,
+                 seed=0):
+    rng = np.random.default_rng(seed)
+    mode = mode_of(dtype)
+    d = 128
+    K = oracle.round_to(rng.standard_normal((P, L, d)) * 0.5, mode).astype(np.float32)
+    V = oracle.round_to(rng.standard_normal((P, L, d)), mode).astype(np.float32)
+    q = oracle.round_to(rng.standard_normal((P, G, d)) * q_scale, mode).astype(np.float32)
+    sel = np.full((P, max(budget, 1)), -1, np.int32)
+    tb = np.zeros(P, np.int32)
+    te = np.zeros(P, np.int32)
+    refs = []
+    for p in range(P):
+        lo, hi = tails[p]
+        tb[p], te[p] = lo, hi
+        cand = np.arange(S, lo)
+        chosen = rng.choice(cand, sel_counts[p], replace=False).astype(np.int32)
+        sel[p, :sel_counts[p]] = chosen
+        rows = oracle.attended_rows(S, chosen, lo, hi)
+        refs.append(oracle.attend(q[p], K[p], V[p], rows, 1 / np.sqrt(d)))
+    dev = cuda_device
+    out = torch.full((P, G, d), float("nan"), device=dev)
+    max_tail = int((te - tb).max())
+    ws = ckv.workspace(ckv.ckv_decode_workspace_bytes(P, G, d, S + budget + max_tail), dev)
+    Kd, Vd = to_dev(K, dtype, dev), to_dev(V, dtype, dev)
+    ckv.ckv_sparse_decode(to_dev(q, dtype, dev), Kd, Vd, Kd.stride(0), L, S,
+                          torch.from_numpy(tb).to(dev), torch.from_numpy(te).to(dev), max_tail,
+                          torch.from_numpy(sel).to(dev),
+                          torch.tensor(sel_counts, dtype=torch.int32, device=dev), budget,
+                          1 / np.sqrt(d), out, ws)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    for p in range(P):
+        err = np.abs(got[p] - refs[p]).max()
+        assert err <= OUT_MAX_ABS, (p, err)
+    assert ckv.ckv_device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("G", [1, 4])
+def test_decode_matches_oracle(cuda_device, dtype, G):
+    _decode_case(cuda_device, dtype, P=5, G=G, L=5000, S=16, sel_counts=[1024, 1000, 0, 1, 777],
+                 tails=[(4936, 5000), (4900, 5000), (4990, 4990), (4000, 4320), (4999, 5000)],
+                 budget=1024, seed=G)
+
+
+def test_decode_peaked_softmax_and_no_rows(cuda_device):
+    # a large query scale makes the softmax peaked (online rescaling matters);
+    # problem 2 attends nothing (no sinks, no recall, empty tail): output 0
+    _decode_case(cuda_device, torch.bfloat16, P=3, G=2, L=3000, S=0, sel_counts=[2048, 5, 0],
+                 tails=[(2900, 3000), (2990, 3000), (2999, 2999)], budget=2048, q_scale=12.0,
+                 seed=7)
