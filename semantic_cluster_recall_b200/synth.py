@@ -60,6 +60,7 @@ class Workload:
     batch: int = 1
     heads_kv: int = 1
     seed: int = 0
+    planted: bool = False  # clustered tokens drawn in M contiguous blocks (test variant)
 
     @property
     def N(self) -> int:
@@ -123,10 +124,13 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
 
 
 def mixture_rows(dirs: torch.Tensor, n: int, sigma: float, g: torch.Generator,
-                 scale: float = 1.0) -> torch.Tensor:
-    """Draw n rows per problem from the mixture with directions dirs [p, M, d] (fp32)."""
+                 scale: float = 1.0, comp: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Draw n rows per problem from the mixture with directions dirs [p, M, d] (fp32).
+
+    comp [p, n] optionally fixes each row's component instead of drawing it."""
     p, M, d = dirs.shape
-    comp = torch.randint(0, M, (p, n), generator=g, device=dirs.device)
+    drawn = torch.randint(0, M, (p, n), generator=g, device=dirs.device)
+    comp = drawn if comp is None else comp
     noise = torch.randn((p, n, d), generator=g, device=dirs.device) * sigma
     x = torch.gather(dirs, 1, comp[..., None].expand(p, n, d)) + noise
     norms = torch.rand((p, n, 1), generator=g, device=dirs.device) * 1.5 + 0.5
@@ -154,10 +158,17 @@ def make_kv(w: Workload, device="cpu", rows: Optional[int] = None,
     dt = w.torch_dtype
     K = out_k if out_k is not None else torch.empty((n, rows, w.d), dtype=dt, device=device)
     V = out_v if out_v is not None else torch.empty((n, rows, w.d), dtype=dt, device=device)
+    comp = None
+    if w.planted:
+        # the clustered rows [S, L - W) come in M equal contiguous blocks, so the
+        # strided seeds land one per block when M divides N (a test variant)
+        comp = torch.randint(0, w.M, (1, rows), device=device)
+        j = torch.arange(w.S, w.L - w.W, device=device)
+        comp[0, w.S:w.L - w.W] = (j - w.S) * w.M // w.N
     for i, p in enumerate(problems):
         dirs = directions(w, p, device)[None]
         gk = _gen(device, w.seed, 2_000_000 + p)
-        K[i] = mixture_rows(dirs, rows, w.sigma, gk)[0].to(dt)
+        K[i] = mixture_rows(dirs, rows, w.sigma, gk, comp=comp)[0].to(dt)
         gv = _gen(device, w.seed, 3_000_000 + p)
         V[i] = torch.randn((rows, w.d), generator=gv, device=device).to(dt)
     return K, V

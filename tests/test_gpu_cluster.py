@@ -60,14 +60,27 @@ def test_cluster_first_divergence_is_a_near_tie(cuda_device, dtype):
 
 
 @pytest.mark.parametrize("G", [1, 4])
-def test_whole_path_on_well_separated_mixture(cuda_device, G):
-    # well separated (small noise) and a peaked query: no near-ties, so the GPU
-    # and the oracle follow the same trajectory and every output can be compared
-    w = small_workload(torch.bfloat16, P=4, G=G, L=6000, C=48, T=5, B=700, M=48,
-                       sigma=0.3 / np.sqrt(128), q_scale=8.0)
+@pytest.mark.parametrize("budget", [100, 6000])
+def test_whole_path_on_planted_mixture(cuda_device, G, budget):
+    # Planted blocks aligned with the strided seeds and small noise: every key's
+    # best centroid wins by a wide margin, so the GPU and the oracle follow the
+    # same trajectory and every output is compared. The query is one
+    # component's direction scaled up, so its own cluster ranks first by a wide
+    # margin; budget 100 recalls part of that cluster only (trimmed), budget
+    # 6000 recalls every clustered token.
+    w = small_workload(torch.bfloat16, P=4, G=G, L=6000, C=40, T=5, B=budget, M=40,
+                       sigma=0.3 / np.sqrt(128)).replace(planted=True)
+    assert w.N % w.C == 0
     K, V = synth.make_kv(w)
-    q = synth.make_queries(w)
-    Kh, Vh, qh = f32np(K), f32np(V), f32np(q)
+    Kh, Vh = f32np(K), f32np(V)
+    rng = np.random.default_rng(G)
+    qh = np.zeros((w.P, G, 128), np.float32)
+    for p in range(w.P):
+        dirs = synth.directions(w, p, "cpu").numpy()
+        for g in range(G):
+            qh[p, g] = dirs[rng.integers(0, w.M)] * 8.0
+    q = torch.from_numpy(qh).to(torch.bfloat16)
+    qh = f32np(q)
     dev = cuda_device
     Kd, Vd, qd = K.to(dev), V.to(dev), q.to(dev)
     st = _run_gpu(Kd, w, w.T, dev)
@@ -82,13 +95,16 @@ def test_whole_path_on_well_separated_mixture(cuda_device, G):
         assert np.array_equal(st.offsets[p, :w.C + 1].cpu().numpy(), r["offsets"])
         assert np.array_equal(st.perm[p, :n].cpu().numpy(), r["perm"])
         assert centroid_rel_err(f32np(st.centroids[p, :w.C]), r["mu"]).max() <= CENT_REL_L2
-        # selection from the GPU's own centroids and the oracle's: compared
-        # through the oracle's scoring of the GPU's scoring copy
-        lp_gpu = f32np(st.centroids_lp[p, :w.C])
-        s = oracle.score(qh[p], lp_gpu)
+        s = oracle.score(qh[p], oracle.round_to(r["mu"], "bf16"))
+        top2 = np.sort(s)[-2:]
         sel, cnt = oracle.select(s, r["offsets"], r["perm"], w.B)
-        assert st.sel_cnt[p].item() == cnt
-        assert np.array_equal(st.sel_idx[p, :cnt].cpu().numpy(), sel)
+        assert st.sel_cnt[p].item() == cnt == min(w.B, n)
+        got = st.sel_idx[p, :cnt].cpu().numpy()
+        if w.B < n:
+            assert top2[1] - top2[0] > 1e-2 * abs(top2[1])  # a clear winner
+            assert np.array_equal(got, sel)
+        else:  # every cluster is recalled: the set is unique, the order is not
+            assert np.array_equal(np.sort(got), np.sort(sel))
         rows = oracle.attended_rows(w.S, sel, w.L - w.W, w.L)
         ref_out = oracle.attend(qh[p], Kh[p], Vh[p], rows, 1 / np.sqrt(128))
         assert np.abs(out[p].cpu().numpy() - ref_out).max() <= OUT_MAX_ABS
