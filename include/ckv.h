@@ -87,6 +87,7 @@ typedef enum { CKV_F32 = 0, CKV_BF16 = 1 } ckv_dtype;
 #define CKV_DEVERR_PERM 0x2u    /* a perm entry outside [tok_begin, tok_end) */
 #define CKV_DEVERR_INDEX 0x4u   /* a selected / tail position outside the K/V rows */
 #define CKV_DEVERR_OFFSETS 0x8u /* offsets not monotone or outside [0, perm_cap] */
+#define CKV_DEVERR_TIMEOUT 0x10u /* a bounded device wait gave up (the kernel stopped early) */
 
 /* Largest supported number of clusters per problem (C_cap). */
 #define CKV_MAX_CLUSTERS 4096
@@ -97,7 +98,9 @@ const char *ckv_last_error(void);
 int ckv_version(void);
 
 /* Read (and optionally clear) the device error word of the current device.
- * Synchronises `stream`. *flags receives the CKV_DEVERR_* bits. */
+ * Synchronises `stream`. *flags receives the CKV_DEVERR_* bits. Returns
+ * CKV_ERR_TIMEOUT if CKV_DEVERR_TIMEOUT is set (the outputs of the call that
+ * set it are incomplete), else CKV_OK. */
 ckv_status ckv_device_error(unsigned int *flags, int clear, void *stream);
 
 /* ---- clustering --------------------------------------------------------- */

@@ -1,0 +1,504 @@
+// a2 assignment for bf16 keys on the sm_100a tensor cores.
+//
+// labels[i] = argmax_c k_i . hat_c: the key-centroid similarity of cosine
+// k-means ("III.B Clustering in the Semantic Space" of "ClusterKV:
+// Manipulating LLM KV Cache in Semantic Space for Recallable Compression",
+// arXiv 2412.03213v2) is a [n x 128] x [128 x C] contraction per problem,
+// followed by a row argmax. The paper runs it with library kernels; here it
+// is one persistent kernel:
+//
+//   warp 4 (1 lane)   TMA producer: 128-key tiles (two 64-column halves,
+//                     128-byte swizzle) into a ring of KST stages, and the
+//                     centroid chunks (resident per problem when they fit in
+//                     shared memory, otherwise streamed through 2 slots)
+//   warp 5 (1 lane)   MMA issuer: tcgen05.mma kind::f16, M = 128 keys,
+//                     N = one centroid chunk (<= 256), K = 128 in 8 steps,
+//                     bf16 x bf16 -> fp32 into one of two TMEM accumulators
+//   warps 0-3         epilogue: each thread owns one key row (TMEM lane),
+//                     reads its accumulator row with tcgen05.ld and keeps a
+//                     running (max, argmax) over the chunks; ties keep the
+//                     lowest centroid index; writes the label
+//
+// Two 256-column TMEM accumulators let the MMA of the next chunk overlap the
+// epilogue of the current one. Tiles are split into contiguous ranges, one
+// per CTA (one CTA per SM), so a CTA reloads resident centroids only when its
+// range crosses into the next problem. Every mbarrier wait is bounded: on
+// timeout the kernel sets CKV_DEVERR_TIMEOUT, stops all roles, waits for its
+// own copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>  // CUtensorMap and its enums (the driver entry point is looked up at run time)
+
+#include "common.cuh"
+
+namespace ckv {
+namespace tc {
+
+constexpr int BM = 128;                          // key rows per tile (MMA M)
+constexpr int KEY_HALF_BYTES = BM * 128;         // 128 rows x 64 bf16
+constexpr int KEY_STAGE_BYTES = 2 * KEY_HALF_BYTES;
+constexpr int ACC_COLS = 256;                    // TMEM columns per accumulator
+constexpr int TMEM_COLS = 512;
+constexpr int NTHREADS = 192;
+constexpr int SMEM_OPTIN_MAX = 232448;           // 227 KB per CTA
+constexpr int SMEM_MIN = 120 * 1024;             // keeps one CTA per SM (TMEM is not shared)
+constexpr unsigned long long TIMEOUT_NS = 2000000000ull;
+constexpr unsigned long long DRAIN_NS = 200000000ull;
+
+struct Args {
+    int n, tok_begin, C, cbase, perm_base, perm_cap;
+    int tpp;             // tiles per problem
+    int total;           // tiles over all problems
+    int nch, ch_rows;    // centroid chunks and rows per chunk (multiple of 16, <= 256)
+    int32_t *labels;
+};
+
+// ---- PTX wrappers ------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of the given parity; false if another role aborted or
+// the wait timed out (then this role raises the abort flag and the error bit).
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > TIMEOUT_NS) {
+            *abort_flag = 1;
+            dev_flag(CKV_DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag (used to drain own async work).
+__device__ __noinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try(bar, parity)) {
+        if (global_ns() - t0 > DRAIN_NS) {
+            dev_flag(CKV_DEVERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), sm_100
+// descriptor version 1. The leading byte offset is unused in this layout.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: D fp32, A and B bf16, both K-major, N and M.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- the kernel ----------------------------------------------------------------
+
+template <bool RESIDENT, int KST>
+__global__ void __launch_bounds__(NTHREADS, 1)
+k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmc,
+            const Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int nslot = RESIDENT ? a.nch : 2;
+    const uint32_t ch_half = (uint32_t)a.ch_rows * 128u;
+    const uint32_t ch_bytes = 2u * ch_half;
+    unsigned char *keys_s = sm;
+    unsigned char *cent_s = sm + KST * KEY_STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(cent_s + (size_t)nslot * ch_bytes);
+    // barrier slots
+    uint64_t *keys_full = bars;                // [KST]
+    uint64_t *keys_empty = bars + KST;         // [KST]
+    uint64_t *cent_full = bars + 2 * KST;      // [2]
+    uint64_t *cent_empty = bars + 2 * KST + 2; // [2]
+    uint64_t *acc_full = bars + 2 * KST + 4;   // [2]
+    uint64_t *acc_empty = bars + 2 * KST + 6;  // [2]
+    uint64_t *drain = bars + 2 * KST + 8;      // [1]
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * KST + 9);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < KST; ++s) {
+            mbar_init(smem_u32(&keys_full[s]), 1);
+            mbar_init(smem_u32(&keys_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&cent_full[s]), 1);
+            mbar_init(smem_u32(&cent_empty[s]), 1);
+            mbar_init(smem_u32(&acc_full[s]), 1);
+            mbar_init(smem_u32(&acc_empty[s]), 4 * 32);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_holder)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int t_begin = (int)((long long)a.total * blockIdx.x / gridDim.x);
+    const int t_end = (int)((long long)a.total * (blockIdx.x + 1) / gridDim.x);
+
+    if (warp == 4) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int last_r[KST];
+            for (int s = 0; s < KST; ++s) last_r[s] = -1;
+            int last_c[2] = {-1, -1};
+            int it = 0, pl = 0, g = 0, cur = -1;
+            bool ok = true;
+            for (int tile = t_begin; tile < t_end && ok; ++tile) {
+                const int p = tile / a.tpp, t = tile - p * a.tpp;
+                if (RESIDENT && p != cur) {
+                    ok = mbar_wait(smem_u32(&cent_empty[0]), (pl & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    const uint32_t fb = smem_u32(&cent_full[0]);
+                    mbar_expect_tx(fb, (uint32_t)a.nch * ch_bytes);
+                    for (int j = 0; j < a.nch; ++j)
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(smem_u32(cent_s + (size_t)j * ch_bytes + h * ch_half), &tmc,
+                                        fb, h * 64, a.cbase + j * a.ch_rows, p);
+                    last_c[0] = pl;
+                    ++pl;
+                    cur = p;
+                }
+                const int s = it % KST, r = it / KST;
+                ok = mbar_wait(smem_u32(&keys_empty[s]), (r & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                const uint32_t kb = smem_u32(&keys_full[s]);
+                mbar_expect_tx(kb, KEY_STAGE_BYTES);
+                for (int h = 0; h < 2; ++h)
+                    tma_load_3d(smem_u32(keys_s + s * KEY_STAGE_BYTES + h * KEY_HALF_BYTES), &tmk,
+                                kb, h * 64, a.tok_begin + t * BM, p);
+                last_r[s] = r;
+                ++it;
+                if (!RESIDENT) {
+                    for (int j = 0; j < a.nch; ++j, ++g) {
+                        const int sl = g & 1, rr = g >> 1;
+                        ok = mbar_wait(smem_u32(&cent_empty[sl]), (rr & 1) ^ 1, abort_flag);
+                        if (!ok) break;
+                        const uint32_t fb = smem_u32(&cent_full[sl]);
+                        mbar_expect_tx(fb, ch_bytes);
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(smem_u32(cent_s + (size_t)sl * ch_bytes + h * ch_half),
+                                        &tmc, fb, h * 64, a.cbase + j * a.ch_rows, p);
+                        last_c[sl] = rr;
+                    }
+                }
+            }
+            // every copy this thread issued has landed before the CTA can exit
+            for (int s = 0; s < KST; ++s)
+                if (last_r[s] >= 0) mbar_drain(smem_u32(&keys_full[s]), last_r[s] & 1);
+            for (int s = 0; s < 2; ++s)
+                if (last_c[s] >= 0) mbar_drain(smem_u32(&cent_full[s]), last_c[s] & 1);
+        }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(BM, a.ch_rows);
+            int it = 0, pl = 0, g = 0, acc = 0, cur = -1;
+            bool ok = true, issued = false;
+            for (int tile = t_begin; tile < t_end && ok; ++tile) {
+                const int p = tile / a.tpp;
+                if (RESIDENT && p != cur) {
+                    ok = mbar_wait(smem_u32(&cent_full[0]), pl & 1, abort_flag);
+                    if (!ok) break;
+                    ++pl;
+                    cur = p;
+                }
+                const int s = it % KST, r = it / KST;
+                ok = mbar_wait(smem_u32(&keys_full[s]), r & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(keys_s + s * KEY_STAGE_BYTES);
+                for (int j = 0; j < a.nch; ++j) {
+                    uint32_t ca;
+                    int sl = 0;
+                    if (RESIDENT) {
+                        ca = smem_u32(cent_s + (size_t)j * ch_bytes);
+                    } else {
+                        sl = g & 1;
+                        ok = mbar_wait(smem_u32(&cent_full[sl]), (g >> 1) & 1, abort_flag);
+                        if (!ok) break;
+                        ca = smem_u32(cent_s + (size_t)sl * ch_bytes);
+                    }
+                    const int buf = acc & 1;
+                    ok = mbar_wait(smem_u32(&acc_empty[buf]), ((acc >> 1) & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + (uint32_t)(buf * ACC_COLS);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t koff = (uint32_t)(k >> 2) * KEY_HALF_BYTES + (k & 3) * 32;
+                        const uint32_t coff = (uint32_t)(k >> 2) * ch_half + (k & 3) * 32;
+                        tc_mma(d, sdesc(ka + koff), sdesc(ca + coff), idesc, k > 0 ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(smem_u32(&acc_full[buf]));
+                    if (!RESIDENT) {
+                        tc_commit(smem_u32(&cent_empty[sl]));
+                        ++g;
+                    }
+                    ++acc;
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&keys_empty[s]));
+                ++it;
+                if (RESIDENT) {
+                    const int nt = tile + 1;
+                    if (nt >= t_end || nt / a.tpp != p) tc_commit(smem_u32(&cent_empty[0]));
+                }
+            }
+            if (issued) {  // all MMAs issued by this thread have completed
+                tc_commit(smem_u32(drain));
+                mbar_drain(smem_u32(drain), 0);
+            }
+        }
+    } else {
+        // ---------------- epilogue: warps 0-3, one key row per thread ----------------
+        const int row_in_tile = warp * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        int acc = 0;
+        bool ok = true;
+        for (int tile = t_begin; tile < t_end && ok; ++tile) {
+            const int p = tile / a.tpp, t = tile - p * a.tpp;
+            float best = -INFINITY;
+            int bidx = 0;
+            for (int j = 0; j < a.nch; ++j) {
+                const int buf = acc & 1;
+                ok = mbar_wait(smem_u32(&acc_full[buf]), (acc >> 1) & 1, abort_flag);
+                ok = __all_sync(FULL, ok);  // tcgen05.ld below needs the whole warp
+                if (!ok) break;
+                tc_fence_after();
+                const int c0 = j * a.ch_rows;
+                const int lim = min(a.ch_rows, a.C - c0);
+                const uint32_t col_base = lane_base + (uint32_t)(buf * ACC_COLS);
+                for (int cc = 0; cc < a.ch_rows; cc += 16) {
+                    float v[16];
+                    tmem_ld16(col_base + cc, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (cc + i < lim && v[i] > best) {
+                            best = v[i];
+                            bidx = c0 + cc + i;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&acc_empty[buf]));
+                ++acc;
+            }
+            if (!ok) break;
+            const int row = t * BM + row_in_tile;
+            if (row < a.n) a.labels[(size_t)p * a.perm_cap + a.perm_base + row] = a.cbase + bidx;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace tc
+
+// ---- host side ---------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        tried = true;
+    }
+    return fn;
+}
+
+// 3-D bf16 tensor map [P][rows][128] with a {64, box_rows, 1} box, 128-byte swizzle.
+inline bool make_map_bf16(CUtensorMap *m, const void *base, int P, long long rows,
+                          long long problem_stride_elems, int box_rows) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)P};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)problem_stride_elems * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct TcPlan {
+    bool resident;
+    int nch, ch_rows;
+    size_t smem;
+};
+
+inline size_t tc_smem_bytes(bool resident, int kst, int nch, int ch_rows) {
+    const size_t slots = resident ? (size_t)nch : 2;
+    size_t s = 1024 /* alignment slack */ + (size_t)kst * tc::KEY_STAGE_BYTES +
+               slots * 2 * (size_t)ch_rows * 128 + 256 /* barriers, TMEM address, flag */;
+    return s < (size_t)tc::SMEM_MIN ? (size_t)tc::SMEM_MIN : s;
+}
+
+inline TcPlan tc_plan(int C) {
+    TcPlan pl;
+    pl.nch = (C + 255) / 256;
+    const int per = (C + pl.nch - 1) / pl.nch;
+    pl.ch_rows = ((per + 15) / 16) * 16;
+    pl.resident = tc_smem_bytes(true, 3, pl.nch, pl.ch_rows) <= (size_t)tc::SMEM_OPTIN_MAX;
+    pl.smem = pl.resident ? tc_smem_bytes(true, 3, pl.nch, pl.ch_rows)
+                          : tc_smem_bytes(false, 2, pl.nch, pl.ch_rows);
+    return pl;
+}
+
+inline ckv_status launch_assign_bf16(const bf16 *keys, int P, int64_t pstride, int tok_begin,
+                                     int n, const bf16 *hat, int C, int cbase, int C_cap,
+                                     int32_t *labels, int perm_base, int perm_cap, int sms,
+                                     cudaStream_t st) {
+    CUtensorMap mk, mc;
+    const TcPlan pl = tc_plan(C);
+    if (!make_map_bf16(&mk, keys, P, pstride / 128, pstride, tc::BM)) return CKV_ERR_CUDA;
+    if (!make_map_bf16(&mc, hat, P, C_cap, (long long)C_cap * 128, pl.ch_rows))
+        return CKV_ERR_CUDA;
+    tc::Args a;
+    a.n = n;
+    a.tok_begin = tok_begin;
+    a.C = C;
+    a.cbase = cbase;
+    a.perm_base = perm_base;
+    a.perm_cap = perm_cap;
+    a.tpp = (n + tc::BM - 1) / tc::BM;
+    a.total = P * a.tpp;
+    a.nch = pl.nch;
+    a.ch_rows = pl.ch_rows;
+    a.labels = labels;
+    const int grid = a.total < sms ? a.total : sms;
+    cudaError_t e;
+    if (pl.resident) {
+        e = cudaFuncSetAttribute(tc::k_assign_tc<true, 3>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+        if (e != cudaSuccess) return CKV_ERR_CUDA;
+        tc::k_assign_tc<true, 3><<<grid, tc::NTHREADS, pl.smem, st>>>(mk, mc, a);
+    } else {
+        e = cudaFuncSetAttribute(tc::k_assign_tc<false, 2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+        if (e != cudaSuccess) return CKV_ERR_CUDA;
+        tc::k_assign_tc<false, 2><<<grid, tc::NTHREADS, pl.smem, st>>>(mk, mc, a);
+    }
+    return cudaGetLastError() == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
+}  // namespace ckv

@@ -10,7 +10,7 @@
 
 #include "common.cuh"
 #include "cluster_kernels.cuh"
-#include "assign_bf16.cuh"
+#include "assign_tc.cuh"
 #include "select_kernels.cuh"
 #include "decode_kernels.cuh"
 
@@ -170,8 +170,12 @@ ckv_status launch_assign(const void *keys, ckv_dtype dt, int P, int64_t pstride,
     if (dt == CKV_F32)
         return launch_assign_f32((const float *)keys, P, pstride, tok_begin, n, (const float *)hat,
                                  C, cbase, C_cap, labels, perm_base, perm_cap, st);
-    return launch_assign_bf16((const bf16 *)keys, P, pstride, tok_begin, n, (const bf16 *)hat, C,
-                              cbase, C_cap, labels, perm_base, perm_cap, st);
+    ckv_status s = launch_assign_bf16((const bf16 *)keys, P, pstride, tok_begin, n,
+                                      (const bf16 *)hat, C, cbase, C_cap, labels, perm_base,
+                                      perm_cap, sm_count(), st);
+    if (s) return fail(s, "tensor-core assignment launch failed (%s)",
+                       cudaGetErrorString(cudaGetLastError()));
+    return ok();
 }
 
 // partial-result slots of the decode workspace (chunks are >= 32 rows)
@@ -225,6 +229,7 @@ ckv_status ckv_device_error(unsigned int *flags, int clear, void *stream) {
     }
     if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
     *flags = v;
+    if (v & CKV_DEVERR_TIMEOUT) return fail(CKV_ERR_TIMEOUT, "a bounded device wait timed out");
     return ok();
 }
 
