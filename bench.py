@@ -436,6 +436,36 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """Run one stage `launches` times on the workload (for profiler captures):
+    the state is prepared by one full clustering first."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    w = synth.WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+    step = Step(w, dev, stream)
+    step.run()
+    st, K = step.st, step.K
+    tb, te = w.S, w.L - w.W
+    calls = {
+        "assign": lambda: ckv.ckv_assign(K, K.stride(0), tb, te, st.centroids_hat, w.C, 0, w.C,
+                                         st.labels, 0, w.N),
+        "index": lambda: ckv.ckv_index(st.labels, w.P, tb, te, w.C, 0, w.C, 0, w.N, st.offsets,
+                                       st.perm, step.ws),
+        "update": lambda: ckv.ckv_update(K, K.stride(0), tb, te, w.C, 0, w.C, st.offsets,
+                                         st.perm, w.N, st.centroids, st.centroids_hat,
+                                         st.centroids_lp, st.sizes),
+        "select": lambda: st.select(step.q),
+        "decode": lambda: st.decode(step.q, step.K, step.V),
+    }
+    for _ in range(args.launches):
+        step.flush_l2()
+        calls[args.only]()
+    torch.cuda.synchronize()
+    print(json.dumps({"only": args.only, "workload": w.name, "launches": args.launches,
+                      "device_error_flags": ckv.ckv_device_error()}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -444,8 +474,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["assign", "index", "update", "select", "decode"],
+                    help="run one stage --launches times (profiler captures); prints no metric")
+    ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -7,17 +7,20 @@
 // followed by a row argmax. The paper runs it with library kernels; here it
 // is one persistent kernel:
 //
-//   warp 4 (1 lane)   TMA producer: 128-key tiles (two 64-column halves,
+//   warp 8 (1 lane)   TMA producer: 128-key tiles (two 64-column halves,
 //                     128-byte swizzle) into a ring of KST stages, and the
 //                     centroid chunks (resident per problem when they fit in
 //                     shared memory, otherwise streamed through 2 slots)
-//   warp 5 (1 lane)   MMA issuer: tcgen05.mma kind::f16, M = 128 keys,
+//   warp 9 (1 lane)   MMA issuer: tcgen05.mma kind::f16, M = 128 keys,
 //                     N = one centroid chunk (<= 256), K = 128 in 8 steps,
 //                     bf16 x bf16 -> fp32 into one of two TMEM accumulators
-//   warps 0-3         epilogue: each thread owns one key row (TMEM lane),
-//                     reads its accumulator row with tcgen05.ld and keeps a
-//                     running (max, argmax) over the chunks; ties keep the
-//                     lowest centroid index; writes the label
+//   warps 0-7         epilogue: warps w and w+4 share TMEM lane quarter w,
+//                     so each key row (TMEM lane) has two threads, each
+//                     reading half of the chunk's columns with tcgen05.ld and
+//                     keeping four independent running (max, argmax) chains
+//                     (instruction-level parallelism); the chains and the two
+//                     halves are merged per tile with ties to the lowest
+//                     centroid index, and the label is written
 //
 // Two 256-column TMEM accumulators let the MMA of the next chunk overlap the
 // epilogue of the current one. Tiles are split into contiguous ranges, one
@@ -39,7 +42,24 @@ constexpr int KEY_HALF_BYTES = BM * 128;         // 128 rows x 64 bf16
 constexpr int KEY_STAGE_BYTES = 2 * KEY_HALF_BYTES;
 constexpr int ACC_COLS = 256;                    // TMEM columns per accumulator
 constexpr int TMEM_COLS = 512;
-constexpr int NTHREADS = 192;
+#ifndef CKV_TC_EPI_PARTS
+#define CKV_TC_EPI_PARTS 4      // epilogue threads per key row
+#endif
+#ifndef CKV_TC_CHAINS
+#define CKV_TC_CHAINS 4         // independent (max, argmax) chains per thread
+#endif
+#ifndef CKV_TC_SUSPEND_NS
+#define CKV_TC_SUSPEND_NS 0     // mbarrier try_wait suspend-time hint (0: none)
+#endif
+constexpr int EPI_PARTS = CKV_TC_EPI_PARTS;
+constexpr int CHAINS = CKV_TC_CHAINS;
+constexpr int EPI_WARPS = 4 * EPI_PARTS;         // EPI_PARTS warps per TMEM lane quarter
+constexpr int MAXG = (16 + EPI_PARTS - 1) / EPI_PARTS;  // 16-column groups per part (chunk <= 256)
+constexpr int PRODUCER_WARP = EPI_WARPS;
+constexpr int MMA_WARP = EPI_WARPS + 1;
+constexpr int NTHREADS = (EPI_WARPS + 2) * 32;
+constexpr int NBAR = 32;                         // mbarrier slots reserved
+constexpr int EPI_SMEM = 2 * (EPI_PARTS - 1) * BM * 8;  // partial results, 2 buffers
 constexpr int SMEM_OPTIN_MAX = 232448;           // 227 KB per CTA
 constexpr int SMEM_MIN = 120 * 1024;             // keeps one CTA per SM (TMEM is not shared)
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;
@@ -74,6 +94,16 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
+#if CKV_TC_SUSPEND_NS > 0
+    // the thread may sleep until the phase completes (or the hint elapses)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"((uint32_t)CKV_TC_SUSPEND_NS)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -81,6 +111,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
@@ -149,19 +180,21 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
+// 16 consecutive fp32 columns of this thread's TMEM lane; the values are
+// valid only after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, float (&v)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+          "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]),
+          "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
         : "r"(taddr)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
@@ -201,8 +234,12 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
     uint64_t *acc_full = bars + 2 * KST + 4;   // [2]
     uint64_t *acc_empty = bars + 2 * KST + 6;  // [2]
     uint64_t *drain = bars + 2 * KST + 8;      // [1]
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * KST + 9);
+    uint64_t *red_full = bars + 2 * KST + 9;   // [2] other parts' partials are written
+    uint64_t *red_empty = bars + 2 * KST + 11; // [2] part 0 has read them
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + NBAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    float *red_v = reinterpret_cast<float *>(bars + NBAR + 1);           // [2][PARTS-1][BM]
+    int *red_i = reinterpret_cast<int *>(red_v + 2 * (EPI_PARTS - 1) * BM);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -214,14 +251,16 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
             mbar_init(smem_u32(&cent_full[s]), 1);
             mbar_init(smem_u32(&cent_empty[s]), 1);
             mbar_init(smem_u32(&acc_full[s]), 1);
-            mbar_init(smem_u32(&acc_empty[s]), 4 * 32);
+            mbar_init(smem_u32(&acc_empty[s]), EPI_WARPS * 32);
+            mbar_init(smem_u32(&red_full[s]), (EPI_PARTS - 1) * 4 * 32 > 0 ? (EPI_PARTS - 1) * 4 * 32 : 1);
+            mbar_init(smem_u32(&red_empty[s]), 4 * 32);
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 5) {
+    if (warp == MMA_WARP) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_holder)),
                      "r"(TMEM_COLS)
@@ -236,7 +275,7 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
     const int t_begin = (int)((long long)a.total * blockIdx.x / gridDim.x);
     const int t_end = (int)((long long)a.total * (blockIdx.x + 1) / gridDim.x);
 
-    if (warp == 4) {
+    if (warp == PRODUCER_WARP) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int last_r[KST];
@@ -289,7 +328,7 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
             for (int s = 0; s < 2; ++s)
                 if (last_c[s] >= 0) mbar_drain(smem_u32(&cent_full[s]), last_c[s] & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == MMA_WARP) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BM, a.ch_rows);
@@ -352,15 +391,24 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
             }
         }
     } else {
-        // ---------------- epilogue: warps 0-3, one key row per thread ----------------
-        const int row_in_tile = warp * 32 + lane;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        int acc = 0;
+        // ------------- epilogue: EPI_PARTS threads per key row (one per warp part) -------------
+        const int quarter = warp & 3, part = warp >> 2;
+        const int row_in_tile = quarter * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const int ngroups = a.ch_rows / 16;               // 16-column groups per chunk
+        const int gper = (ngroups + EPI_PARTS - 1) / EPI_PARTS;  // <= MAXG
+        const int g_lo = min(ngroups, part * gper), g_hi = min(ngroups, g_lo + gper);
+        int acc = 0, nt = 0;
         bool ok = true;
-        for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        for (int tile = t_begin; tile < t_end && ok; ++tile, ++nt) {
             const int p = tile / a.tpp, t = tile - p * a.tpp;
-            float best = -INFINITY;
-            int bidx = 0;
+            float best[CHAINS];
+            int bidx[CHAINS];
+#pragma unroll
+            for (int k = 0; k < CHAINS; ++k) {
+                best[k] = -INFINITY;
+                bidx[k] = 0x7fffffff;
+            }
             for (int j = 0; j < a.nch; ++j) {
                 const int buf = acc & 1;
                 ok = mbar_wait(smem_u32(&acc_full[buf]), (acc >> 1) & 1, abort_flag);
@@ -368,32 +416,88 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
                 if (!ok) break;
                 tc_fence_after();
                 const int c0 = j * a.ch_rows;
-                const int lim = min(a.ch_rows, a.C - c0);
+                const int lim = min(a.ch_rows, a.C - c0);  // valid columns of this chunk
                 const uint32_t col_base = lane_base + (uint32_t)(buf * ACC_COLS);
-                for (int cc = 0; cc < a.ch_rows; cc += 16) {
-                    float v[16];
-                    tmem_ld16(col_base + cc, v);
+                // copy this thread's slice of the chunk to registers and hand the
+                // accumulator back to the MMA warp at once; the argmax runs after
+                float v[MAXG][16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        if (cc + i < lim && v[i] > best) {
-                            best = v[i];
-                            bidx = c0 + cc + i;
+                for (int u = 0; u < MAXG; ++u)
+                    if (g_lo + u < g_hi) tmem_ld16_nowait(col_base + (g_lo + u) * 16, v[u]);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&acc_empty[buf]));
+#pragma unroll
+                for (int u = 0; u < MAXG; ++u) {
+                    const int gc = (g_lo + u) * 16;
+                    if (g_lo + u < g_hi && gc < lim) {
+                        if (gc + 16 <= lim) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int k = (u * 16 + i) % CHAINS;
+                                const bool take = v[u][i] > best[k];
+                                best[k] = take ? v[u][i] : best[k];
+                                bidx[k] = take ? c0 + gc + i : bidx[k];
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int k = (u * 16 + i) % CHAINS;
+                                const bool take = (gc + i < lim) && v[u][i] > best[k];
+                                best[k] = take ? v[u][i] : best[k];
+                                bidx[k] = take ? c0 + gc + i : bidx[k];
+                            }
                         }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(smem_u32(&acc_empty[buf]));
                 ++acc;
             }
             if (!ok) break;
-            const int row = t * BM + row_in_tile;
-            if (row < a.n) a.labels[(size_t)p * a.perm_cap + a.perm_base + row] = a.cbase + bidx;
+            // merge the chains: larger value, then lower index
+            float bv = best[0];
+            int bi = bidx[0];
+#pragma unroll
+            for (int k = 1; k < CHAINS; ++k)
+                if (best[k] > bv || (best[k] == bv && bidx[k] < bi)) {
+                    bv = best[k];
+                    bi = bidx[k];
+                }
+            // merge the parts of the row (bounded mbarrier handshake)
+            const int rb = nt & 1;
+            if (part > 0) {
+                ok = mbar_wait(smem_u32(&red_empty[rb]), ((nt >> 1) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                const int slot = (rb * (EPI_PARTS - 1) + part - 1) * BM + row_in_tile;
+                red_v[slot] = bv;
+                red_i[slot] = bi;
+                mbar_arrive(smem_u32(&red_full[rb]));
+            } else {
+                if (EPI_PARTS > 1) {
+                    ok = mbar_wait(smem_u32(&red_full[rb]), (nt >> 1) & 1, abort_flag);
+                    if (!ok) break;
+#pragma unroll
+                    for (int q = 1; q < EPI_PARTS; ++q) {
+                        const int slot = (rb * (EPI_PARTS - 1) + q - 1) * BM + row_in_tile;
+                        const float ov = red_v[slot];
+                        const int oi = red_i[slot];
+                        if (ov > bv || (ov == bv && oi < bi)) {
+                            bv = ov;
+                            bi = oi;
+                        }
+                    }
+                    mbar_arrive(smem_u32(&red_empty[rb]));
+                }
+                const int row = t * BM + row_in_tile;
+                if (bi == 0x7fffffff) bi = 0;  // no valid column (cannot happen for C >= 1)
+                if (row < a.n)
+                    a.labels[(size_t)p * a.perm_cap + a.perm_base + row] = a.cbase + bi;
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == MMA_WARP) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(TMEM_COLS)
@@ -449,7 +553,8 @@ struct TcPlan {
 inline size_t tc_smem_bytes(bool resident, int kst, int nch, int ch_rows) {
     const size_t slots = resident ? (size_t)nch : 2;
     size_t s = 1024 /* alignment slack */ + (size_t)kst * tc::KEY_STAGE_BYTES +
-               slots * 2 * (size_t)ch_rows * 128 + 256 /* barriers, TMEM address, flag */;
+               slots * 2 * (size_t)ch_rows * 128 + tc::NBAR * 8 + 8 /* TMEM address, flag */ +
+               tc::EPI_SMEM;
     return s < (size_t)tc::SMEM_MIN ? (size_t)tc::SMEM_MIN : s;
 }
 

@@ -292,9 +292,33 @@ k_index_scatter(const int32_t *__restrict__ labels, int perm_base, int perm_cap,
 
 // ---------------------------------------------------------------------------
 // a3 centroid update: one warp per cluster gathers its member rows through
-// perm (256-byte rows for bf16), sums them in fp32 in perm order, divides by
-// the count and renormalises. Deterministic: no atomics.
+// perm. A 16-lane half-warp owns one row at a time (16 bytes per lane for
+// bf16, i.e. a whole 256-byte row per half-warp) and keeps 8 rows in flight;
+// the two halves take alternate rows and are added at the end. Sums are fp32,
+// in a fixed order (deterministic, no atomics); then the mean, its norm, and
+// the two rounded copies.
 // ---------------------------------------------------------------------------
+constexpr int UPD_ROWS = 8;  // rows in flight per half-warp
+
+template <typename T>
+__device__ __forceinline__ void store8(T *p, const float (&v)[8]);
+
+template <>
+__device__ __forceinline__ void store8<float>(float *p, const float (&v)[8]) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <>
+__device__ __forceinline__ void store8<bf16>(bf16 *p, const float (&v)[8]) {
+    uint4 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    u.z = pack_bf16x2(v[4], v[5]);
+    u.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(p) = u;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end, int C,
@@ -302,6 +326,7 @@ k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end
          const int32_t *__restrict__ perm, int perm_cap, float *__restrict__ cent,
          T *__restrict__ hat, T *__restrict__ lp, int32_t *__restrict__ sizes) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = lane >> 4, hl = lane & 15;
     const int c = blockIdx.x * 8 + warp;
     const int p = blockIdx.y;
     if (c >= C) return;
@@ -315,45 +340,61 @@ k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end
         }
         return;
     }
-    const T *kb = keys + (int64_t)p * pstride + lane * 4;
+    const T *kb = keys + (int64_t)p * pstride + hl * 8;
     const int32_t *pp = perm + (size_t)p * perm_cap;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
     for (int j0 = o0; j0 < o1; j0 += 32) {
         const int cnt = min(32, o1 - j0);
         const int pos = lane < cnt ? pp[j0 + lane] : -1;
-        for (int k = 0; k < cnt; k += 4) {
-            float4 v[4];
+        for (int k = 0; k < cnt; k += 2 * UPD_ROWS) {
+            Row8<T> r[UPD_ROWS];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int kk = k + u;
+            for (int u = 0; u < UPD_ROWS; ++u) {
+                const int kk = k + 2 * u + half;  // < 32 always
                 const int ps = __shfl_sync(FULL, pos, kk & 31);
-                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                r[u].zero();
                 if (kk < cnt) {
-                    if (ps >= tok_begin && ps < tok_end) v[u] = load4(kb + (int64_t)ps * D);
-                    else if (lane == 0) dev_flag(CKV_DEVERR_PERM);
+                    if (ps >= tok_begin && ps < tok_end) r[u].load(kb + (int64_t)ps * D);
+                    else if (hl == 0) dev_flag(CKV_DEVERR_PERM);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                acc.x += v[u].x;
-                acc.y += v[u].y;
-                acc.z += v[u].z;
-                acc.w += v[u].w;
+            for (int u = 0; u < UPD_ROWS; ++u) {
+                float f[8];
+                r[u].to_float(f);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[t] += f[t];
             }
         }
     }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(FULL, acc[t], 16);
     const int n = o1 - o0;
     if (lane == 0) *sz = n;
     if (n == 0) return;
     const float fn = (float)n;
-    float4 mu = make_float4(acc.x / fn, acc.y / fn, acc.z / fn, acc.w / fn);
-    const float ss = warp_sum(mu.x * mu.x + mu.y * mu.y + mu.z * mu.z + mu.w * mu.w);
+    float mu[8];
+    float ss = 0.f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        mu[t] = acc[t] / fn;
+        ss = fmaf(mu[t], mu[t], ss);
+    }
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
     if (!(ss > 0.f)) return;
-    const float nrm = sqrtf(ss);
-    const size_t o = ((size_t)p * C_cap + cbase + c) * D + lane * 4;
-    store4(cent + o, mu);
-    store4(lp + o, mu);
-    store4(hat + o, make_float4(mu.x / nrm, mu.y / nrm, mu.z / nrm, mu.w / nrm));
+    if (half == 0) {
+        const float nrm = sqrtf(ss);
+        float h[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) h[t] = mu[t] / nrm;
+        const size_t o = ((size_t)p * C_cap + cbase + c) * D + hl * 8;
+        store8<float>(cent + o, mu);
+        store8<T>(lp + o, mu);
+        store8<T>(hat + o, h);
+    }
 }
 
 }  // namespace ckv
