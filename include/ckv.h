@@ -221,6 +221,39 @@ ckv_status ckv_sparse_decode(const void *q, const void *K, const void *V, ckv_dt
                              float scale, float *out, void *workspace, size_t ws_bytes,
                              void *stream);
 
+/* Allocation-free variant of ckv_sparse_decode. The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory --
+ * a plugin or operator hook that is handed its tensors by a host framework
+ * but no allocator (the framework's pool owns the device memory, so a private
+ * cudaMalloc would bypass its accounting or fail once the pool has reserved
+ * the device), and decode loops that must not call cudaMalloc/cudaFree at all
+ * because those calls can synchronise the device and stall other streams.
+ * Such a caller still passes q, K, V, the selection and `out` exactly as for
+ * ckv_sparse_decode, but no workspace: the split-K partials live in a fixed
+ * file-scope device array of CKV_NOALLOC_SCRATCH_BYTES inside the library
+ * (one per GPU that loads the library, held until the process exits).
+ *   - A call whose partials would not fit returns CKV_ERR_INVALID with a
+ *     clear message and launches nothing; ckv_sparse_decode_noalloc_scratch_bytes
+ *     gives the bytes a shape needs on the current device.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents (nothing in it needs to start at zero: each call writes
+ *     every partial it reads). Calls that overlap on the GPU (other streams,
+ *     other host threads) race on it: serialise them.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ * Arguments, layout, results and errors are otherwise those of
+ * ckv_sparse_decode. */
+#define CKV_NOALLOC_SCRATCH_BYTES (8u << 20)
+size_t ckv_sparse_decode_noalloc_scratch_bytes(int P, int G, int d, int max_rows);
+ckv_status ckv_sparse_decode_noalloc(const void *q, const void *K, const void *V, ckv_dtype dt,
+                                     int P, int G, int d, int64_t kv_problem_stride,
+                                     int kv_rows, int sink, const int32_t *tail_begin,
+                                     const int32_t *tail_end, int max_tail,
+                                     const int32_t *sel_idx, const int32_t *sel_cnt,
+                                     int budget, float scale, float *out, void *stream);
+
 /* Append one generated token per problem: K/V row tail_end[p] <- new_k[p] /
  * new_v[p] (dtype [P][d]); then tail_end[p] += 1. A full cache (tail_end[p]
  * >= kv_rows) writes nothing and sets CKV_DEVERR_INDEX. */

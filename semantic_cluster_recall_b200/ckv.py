@@ -29,7 +29,9 @@ EXPORTS = [
     "ckv_init_centroids", "ckv_assign", "ckv_index", "ckv_update",
     "ckv_select_workspace_bytes", "ckv_select",
     "ckv_decode_workspace_bytes", "ckv_sparse_decode", "ckv_append",
+    "ckv_sparse_decode_noalloc_scratch_bytes", "ckv_sparse_decode_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class CkvError(RuntimeError):
@@ -81,6 +83,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "ckv_sparse_decode": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, vp, vp, i32,
                                     vp, vp, i32, f32, vp, vp, sz, vp]),
         "ckv_append": (i32, [vp, vp, i32, i32, i32, i64, i32, vp, vp, vp, vp]),
+        "ckv_sparse_decode_noalloc_scratch_bytes": (sz, [i32, i32, i32, i32]),
+        "ckv_sparse_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, vp,
+                                            vp, i32, vp, vp, i32, f32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -211,6 +216,26 @@ def ckv_sparse_decode(q, K, V, kv_problem_stride, kv_rows, sink, tail_begin, tai
                                   _p(sel_idx), _p(sel_cnt), budget, float(scale), _p(out), _p(ws),
                                   ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "ckv_sparse_decode")
+
+
+def ckv_sparse_decode_noalloc(q, K, V, kv_problem_stride, kv_rows, sink, tail_begin, tail_end,
+                              max_tail, sel_idx, sel_cnt, budget, scale, out, P=None, G=None,
+                              d=128, stream=None):
+    """ckv_sparse_decode without a workspace, for callers that cannot allocate
+    device memory: the library's fixed scratch array holds the partials (see
+    include/ckv.h for the size limit and for the rule that overlapping calls
+    race on that array)."""
+    P = q.shape[0] if P is None else P
+    G = q.shape[1] if G is None else G
+    st = load().ckv_sparse_decode_noalloc(_p(q), _p(K), _p(V), dtype_code(q), P, G, d,
+                                          kv_problem_stride, kv_rows, sink, _p(tail_begin),
+                                          _p(tail_end), max_tail, _p(sel_idx), _p(sel_cnt),
+                                          budget, float(scale), _p(out), _stream(stream))
+    _check(st, "ckv_sparse_decode_noalloc")
+
+
+def ckv_sparse_decode_noalloc_scratch_bytes(P: int, G: int, d: int, max_rows: int) -> int:
+    return int(load().ckv_sparse_decode_noalloc_scratch_bytes(P, G, d, max_rows))
 
 
 def ckv_append(K, V, kv_problem_stride, kv_rows, new_k, new_v, tail_end, P=None, d=128,

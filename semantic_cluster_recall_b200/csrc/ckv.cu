@@ -502,3 +502,118 @@ ckv_status ckv_append(void *K, void *V, ckv_dtype dt, int P, int d, int64_t kv_p
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free sparse decode: the split-K partials live in a fixed array
+// inside the library instead of a caller workspace. See ckv.h
+// (ckv_sparse_decode_noalloc) for who needs this and its limits.
+// ---------------------------------------------------------------------------
+
+// One copy per device that loads the library, held until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_decode_scratch[CKV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[MAX_DEVICES] = {nullptr};
+
+// Device address of the fixed scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+ckv_status noalloc_scratch(void **addr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= MAX_DEVICES) return fail(CKV_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_decode_scratch);
+        if (e != cudaSuccess || !ptr)
+            return fail(CKV_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        g_noalloc_addr[dev] = ptr;
+    }
+    *addr = g_noalloc_addr[dev];
+    return CKV_OK;
+}
+
+}  // namespace
+
+extern "C" size_t ckv_sparse_decode_noalloc_scratch_bytes(int P, int G, int d, int max_rows) {
+    if (P < 1 || G < 1 || d != D) return 0;
+    int chunk, nsplit;
+    decode_shape(P, max_rows, sm_count(), &chunk, &nsplit);
+    const size_t parts = (size_t)P * nsplit * G;
+    return align256(parts * D * sizeof(float)) + align256(parts * sizeof(float2));
+}
+
+extern "C" ckv_status ckv_sparse_decode_noalloc(const void *q, const void *K, const void *V,
+                                                ckv_dtype dt, int P, int G, int d,
+                                                int64_t kv_problem_stride, int kv_rows, int sink,
+                                                const int32_t *tail_begin,
+                                                const int32_t *tail_end, int max_tail,
+                                                const int32_t *sel_idx, const int32_t *sel_cnt,
+                                                int budget, float scale, float *out,
+                                                void *stream) {
+    if (!q || !K || !V || !tail_begin || !tail_end || !sel_cnt || !out)
+        return fail(CKV_ERR_INVALID, "null pointer argument");
+    if (budget > 0 && !sel_idx) return fail(CKV_ERR_INVALID, "sel_idx is null");
+    if (!valid_dtype(dt)) return fail(CKV_ERR_INVALID, "unknown dtype %d", (int)dt);
+    if (d != D) return fail(CKV_ERR_INVALID, "d must be 128 (got %d)", d);
+    if (P < 1 || P > 65535) return fail(CKV_ERR_INVALID, "bad P %d", P);
+    if (G < 1 || G > 8 || (G & (G - 1)))
+        return fail(CKV_ERR_INVALID, "G must be 1, 2, 4 or 8 (got %d)", G);
+    if (kv_rows < 1 || kv_problem_stride < (int64_t)kv_rows * D)
+        return fail(CKV_ERR_INVALID, "kv_problem_stride < kv_rows * d");
+    if (sink < 0 || sink > kv_rows) return fail(CKV_ERR_INVALID, "bad sink %d", sink);
+    if (budget < 0 || max_tail < 0) return fail(CKV_ERR_INVALID, "negative budget or max_tail");
+    if (!(scale > 0.f) || !isfinite(scale)) return fail(CKV_ERR_INVALID, "bad scale");
+    const size_t esz = dt == CKV_BF16 ? 2 : 4;
+    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) ||
+        ((size_t)kv_problem_stride * esz) % 16)
+        return fail(CKV_ERR_INVALID, "q, K, V and the problem stride must be 16-byte aligned");
+    const int64_t max_rows64 = (int64_t)sink + budget + max_tail;
+    if (max_rows64 > (1 << 30)) return fail(CKV_ERR_INVALID, "too many attended rows");
+    const int max_rows = (int)max_rows64;
+    int chunk, nsplit;
+    decode_shape(P, max_rows, sm_count(), &chunk, &nsplit);
+    const size_t parts = (size_t)P * nsplit * G;
+    const size_t o_bytes = align256(parts * D * sizeof(float));
+    const size_t need = o_bytes + align256(parts * sizeof(float2));
+    if (need > (size_t)CKV_NOALLOC_SCRATCH_BYTES)
+        return fail(CKV_ERR_INVALID,
+                    "this decode needs %zu bytes of scratch, more than the fixed %zu bytes of "
+                    "ckv_sparse_decode_noalloc; use ckv_sparse_decode with a workspace",
+                    need, (size_t)CKV_NOALLOC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    ckv_status s = noalloc_scratch(&scratch);
+    if (s) return s;
+    float *part_o = reinterpret_cast<float *>(scratch);
+    float2 *part_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(scratch) + o_bytes);
+    const float qscale = scale * 1.4426950408889634f;
+    cudaStream_t st = S(stream);
+    dim3 grid(nsplit, P);
+#define CKV_DEC_NA(T, GG)                                                                        \
+    do {                                                                                         \
+        k_decode_split<T, GG><<<grid, DEC_THREADS, 0, st>>>(                                     \
+            (const T *)q, (const T *)K, (const T *)V, kv_problem_stride, kv_rows, sink,          \
+            tail_begin, tail_end, sel_idx, sel_cnt, budget, qscale, chunk, nsplit, part_o,       \
+            part_ml);                                                                            \
+        k_decode_combine<GG><<<P, D, 0, st>>>(part_o, part_ml, nsplit, out);                     \
+    } while (0)
+#define CKV_DEC_NA_G(T)                     \
+    switch (G) {                            \
+        case 1: CKV_DEC_NA(T, 1); break;    \
+        case 2: CKV_DEC_NA(T, 2); break;    \
+        case 4: CKV_DEC_NA(T, 4); break;    \
+        default: CKV_DEC_NA(T, 8); break;   \
+    }
+    if (dt == CKV_BF16) {
+        CKV_DEC_NA_G(bf16)
+    } else {
+        CKV_DEC_NA_G(float)
+    }
+#undef CKV_DEC_NA_G
+#undef CKV_DEC_NA
+    return launched("k_decode (noalloc)");
+}
