@@ -177,7 +177,7 @@ class Step:
         st.tail_begin.fill_(w.L - w.W)
         st.tail_end.fill_(w.L)
         self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-        self.launches_per_step = 1 + w.T * 5 + 2 + 2
+        self.launches_per_step = 1 + w.T * 5 + (1 if w.G in (1, 2, 4) else 4)
 
     def run(self, ev_assign=None, ev_decode=None):
         w, st, K = self.w, self.st, self.K
@@ -198,8 +198,7 @@ class Step:
                            stream=self.stream)
         if ev_decode is not None:
             ev_decode[0].record(self.stream)
-        st.select(self.q)
-        st.decode(self.q, self.K, self.V)
+        st.step(self.q, self.K, self.V)
         if ev_decode is not None:
             ev_decode[1].record(self.stream)
 
@@ -208,18 +207,28 @@ class Step:
 
 
 def time_decode_steps(step: Step, n: int):
-    """Decode steps alone (select + sparse decode), each with L2 flushed first."""
+    """Decode steps alone (select + sparse decode), each with L2 flushed first.
+
+    The step's launches are captured once in a CUDA graph and replayed, so the
+    time is the device's (no per-launch host overhead between the kernels)."""
+    st, s = step.st, step.stream
+    st.step(step.q, step.K, step.V)  # warm-up outside the capture (one-time set-up)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        st.step(step.q, step.K, step.V)
+    torch.cuda.synchronize()
     times = []
     for i in range(n):
         step.flush_l2()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record(step.stream)
-        step.st.select(step.q)
-        step.st.decode(step.q, step.K, step.V)
-        b.record(step.stream)
+        a.record(s)
+        g.replay()
+        b.record(s)
         b.synchronize()
         times.append(a.elapsed_time(b) * 1e-3)
+    del g
     return times
 
 
@@ -374,7 +383,8 @@ def run_ours(args):
                                 "peak": pk["hbm_gbs"], "unit": "GB/s",
                                 "frac": dec_bytes / t_dec / 1e9 / pk["hbm_gbs"],
                                 "peak_source": pk["source"] + " copy"},
-                   "l2": "flushed before every decode step"},
+                   "l2": "flushed before every decode step",
+                   "launch": "fused select + sparse decode (one cluster launch), CUDA graph replay"},
         "e2e": {"value": world * keys / e2e_s, "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
         "gpu_launches": launches,
@@ -457,6 +467,7 @@ def run_only(args):
                                          st.centroids_lp, st.sizes),
         "select": lambda: st.select(step.q),
         "decode": lambda: st.decode(step.q, step.K, step.V),
+        "step": lambda: st.step(step.q, step.K, step.V),
     }
     for _ in range(args.launches):
         step.flush_l2()
@@ -474,7 +485,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["assign", "index", "update", "select", "decode"],
+    ap.add_argument("--only", choices=["assign", "index", "update", "select", "decode", "step"],
                     help="run one stage --launches times (profiler captures); prints no metric")
     ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()

@@ -197,6 +197,25 @@ ckv_status ckv_select(const void *q, ckv_dtype dt, int P, int G, int d,
                       int32_t *sel_idx, int32_t *sel_cnt, void *workspace, size_t ws_bytes,
                       void *stream);
 
+/* ---- fused decode step -------------------------------------------------- */
+
+/* One decode step in one launch: ckv_select followed by ckv_sparse_decode,
+ * with the same arguments, outputs and results (sel_idx / sel_cnt
+ * bit-identical to ckv_select; out equal to ckv_sparse_decode up to fp32
+ * summation order). One thread-block cluster of up to 8 CTAs per problem
+ * shares the scores, ranks and partial attention results through
+ * distributed shared memory, so no workspace and no second kernel are
+ * needed. Supports G in {1, 2, 4} and up to 32768 attended rows per problem
+ * (sink + budget + max_tail); other shapes return CKV_ERR_UNSUPPORTED (use
+ * the two separate calls). */
+ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
+                             const void *centroids_lp, const int32_t *n_clusters, int C_cap,
+                             const int32_t *offsets, const int32_t *perm, int perm_cap,
+                             int budget, int32_t *sel_idx, int32_t *sel_cnt, const void *K,
+                             const void *V, int64_t kv_problem_stride, int kv_rows, int sink,
+                             const int32_t *tail_begin, const int32_t *tail_end, int max_tail,
+                             float scale, float *out, void *stream);
+
 /* ---- sparse decode attention -------------------------------------------- */
 
 /* max_rows bounds sink + budget + (tail_end - tail_begin) over all problems. */

@@ -30,6 +30,7 @@ EXPORTS = [
     "ckv_select_workspace_bytes", "ckv_select",
     "ckv_decode_workspace_bytes", "ckv_sparse_decode", "ckv_append",
     "ckv_sparse_decode_noalloc_scratch_bytes", "ckv_sparse_decode_noalloc",
+    "ckv_select_decode",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -84,6 +85,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
                                     vp, vp, i32, f32, vp, vp, sz, vp]),
         "ckv_append": (i32, [vp, vp, i32, i32, i32, i64, i32, vp, vp, vp, vp]),
         "ckv_sparse_decode_noalloc_scratch_bytes": (sz, [i32, i32, i32, i32]),
+        "ckv_select_decode": (i32, [vp, i32, i32, i32, i32, vp, vp, i32, vp, vp, i32, i32, vp, vp,
+                                    vp, vp, i64, i32, i32, vp, vp, i32, f32, vp, vp]),
         "ckv_sparse_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, vp,
                                             vp, i32, vp, vp, i32, f32, vp, vp]),
     }
@@ -204,6 +207,19 @@ def ckv_select(q, centroids_lp, n_clusters, C_cap, offsets, perm, perm_cap, budg
                            C_cap, _p(offsets), _p(perm), perm_cap, budget, _p(sel_idx),
                            _p(sel_cnt), _p(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "ckv_select")
+
+
+def ckv_select_decode(q, centroids_lp, n_clusters, C_cap, offsets, perm, perm_cap, budget,
+                      sel_idx, sel_cnt, K, V, kv_problem_stride, kv_rows, sink, tail_begin,
+                      tail_end, max_tail, scale, out, P=None, G=None, d=128, stream=None):
+    P = q.shape[0] if P is None else P
+    G = q.shape[1] if G is None else G
+    st = load().ckv_select_decode(_p(q), dtype_code(q), P, G, d, _p(centroids_lp),
+                                  _p(n_clusters), C_cap, _p(offsets), _p(perm), perm_cap, budget,
+                                  _p(sel_idx), _p(sel_cnt), _p(K), _p(V), kv_problem_stride,
+                                  kv_rows, sink, _p(tail_begin), _p(tail_end), max_tail,
+                                  float(scale), _p(out), _stream(stream))
+    _check(st, "ckv_select_decode")
 
 
 def ckv_sparse_decode(q, K, V, kv_problem_stride, kv_rows, sink, tail_begin, tail_end, max_tail,

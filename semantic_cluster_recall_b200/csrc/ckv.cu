@@ -13,6 +13,7 @@
 #include "assign_tc.cuh"
 #include "select_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "select_decode.cuh"
 
 using namespace ckv;
 
@@ -79,7 +80,8 @@ cudaError_t smem_optin(K kernel, size_t bytes, int slot) {
 }
 
 // slots for smem_optin (one per kernel instantiation that may exceed 48 KB)
-enum { SLOT_ASSIGN_F32 = 0, SLOT_ASSIGN_BF16, SLOT_HIST, SLOT_SCATTER, SLOT_RANK, SLOT_ASSIGN_TC };
+enum { SLOT_ASSIGN_F32 = 0, SLOT_ASSIGN_BF16, SLOT_HIST, SLOT_SCATTER, SLOT_RANK, SLOT_ASSIGN_TC,
+       SLOT_SD_BASE /* + 6 fused select-decode instantiations */ };
 
 bool valid_dtype(ckv_dtype dt) { return dt == CKV_F32 || dt == CKV_BF16; }
 
@@ -406,6 +408,97 @@ ckv_status ckv_select(const void *q, ckv_dtype dt, int P, int G, int d, const vo
     k_rankfill<<<P, 1024, smem, st>>>(scores, n_clusters, C_cap, offsets, perm, perm_cap, budget,
                                        sel_idx, sel_cnt);
     return launched("k_rankfill");
+}
+
+ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
+                             const void *centroids_lp, const int32_t *n_clusters, int C_cap,
+                             const int32_t *offsets, const int32_t *perm, int perm_cap,
+                             int budget, int32_t *sel_idx, int32_t *sel_cnt, const void *K,
+                             const void *V, int64_t kv_problem_stride, int kv_rows, int sink,
+                             const int32_t *tail_begin, const int32_t *tail_end, int max_tail,
+                             float scale, float *out, void *stream) {
+    if (!q || !centroids_lp || !n_clusters || !offsets || !perm || !sel_cnt || !K || !V ||
+        !tail_begin || !tail_end || !out)
+        return fail(CKV_ERR_INVALID, "null pointer argument");
+    if (budget > 0 && !sel_idx) return fail(CKV_ERR_INVALID, "sel_idx is null");
+    if (!valid_dtype(dt)) return fail(CKV_ERR_INVALID, "unknown dtype %d", (int)dt);
+    if (d != D) return fail(CKV_ERR_INVALID, "d must be 128 (got %d)", d);
+    if (P < 1 || P > 65535) return fail(CKV_ERR_INVALID, "bad P %d", P);
+    if (G != 1 && G != 2 && G != 4)
+        return fail(CKV_ERR_UNSUPPORTED, "fused step supports G = 1, 2, 4 (got %d)", G);
+    if (C_cap < 1 || C_cap > CKV_MAX_CLUSTERS) return fail(CKV_ERR_INVALID, "bad C_cap %d", C_cap);
+    if (perm_cap < 1) return fail(CKV_ERR_INVALID, "bad perm_cap %d", perm_cap);
+    if (budget < 0 || max_tail < 0) return fail(CKV_ERR_INVALID, "negative budget or max_tail");
+    if (kv_rows < 1 || kv_problem_stride < (int64_t)kv_rows * D)
+        return fail(CKV_ERR_INVALID, "kv_problem_stride < kv_rows * d");
+    if (sink < 0 || sink > kv_rows) return fail(CKV_ERR_INVALID, "bad sink %d", sink);
+    if (!(scale > 0.f) || !isfinite(scale)) return fail(CKV_ERR_INVALID, "bad scale");
+    const size_t esz = dt == CKV_BF16 ? 2 : 4;
+    if (!aligned(q, 16) || !aligned(centroids_lp, 16) || !aligned(K, 16) || !aligned(V, 16) ||
+        ((size_t)kv_problem_stride * esz) % 16)
+        return fail(CKV_ERR_INVALID, "q, centroids_lp, K, V and the problem stride must be 16-byte aligned");
+    const int64_t max_rows64 = (int64_t)sink + budget + max_tail;
+    if (max_rows64 > (1 << 30)) return fail(CKV_ERR_INVALID, "too many attended rows");
+    const int max_rows = max_rows64 < 1 ? 1 : (int)max_rows64;
+    const int sms = sm_count();
+    int nc = (4 * sms + P - 1) / P;
+    nc = nc < 1 ? 1 : (nc > sd::NC_MAX ? sd::NC_MAX : nc);
+    int chunk = (max_rows + nc - 1) / nc;
+    if (chunk > sd::POS_MAX)
+        return fail(CKV_ERR_UNSUPPORTED, "fused step supports up to %d attended rows per problem",
+                    sd::NC_MAX * sd::POS_MAX);
+    const size_t smem = sd::layout(C_cap, G, chunk, nc).total;
+    sd::Args a;
+    a.q = q;
+    a.lp = centroids_lp;
+    a.ncl = n_clusters;
+    a.C_cap = C_cap;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.perm_cap = perm_cap;
+    a.B = budget;
+    a.K = K;
+    a.V = V;
+    a.kvs = kv_problem_stride;
+    a.kv_rows = kv_rows;
+    a.S = sink;
+    a.tail_b = tail_begin;
+    a.tail_e = tail_end;
+    a.qscale = scale * 1.4426950408889634f;
+    a.chunk = chunk;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.out = out;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nc, P, 1);
+    cfg.blockDim = dim3(sd::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = S(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaSuccess;
+#define CKV_SD(T, GG)                                                                     \
+    do {                                                                                  \
+        e = smem_optin(sd::k_select_decode<T, GG>, smem, SLOT_SD_BASE + (sizeof(T) == 2) * 3 + (GG == 1 ? 0 : GG == 2 ? 1 : 2)); \
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sd::k_select_decode<T, GG>, a); \
+    } while (0)
+    if (dt == CKV_BF16) {
+        if (G == 1) CKV_SD(bf16, 1);
+        else if (G == 2) CKV_SD(bf16, 2);
+        else CKV_SD(bf16, 4);
+    } else {
+        if (G == 1) CKV_SD(float, 1);
+        else if (G == 2) CKV_SD(float, 2);
+        else CKV_SD(float, 4);
+    }
+#undef CKV_SD
+    if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "k_select_decode: %s", cudaGetErrorString(e));
+    return launched("k_select_decode");
 }
 
 size_t ckv_decode_workspace_bytes(int P, int G, int d, int max_rows) {

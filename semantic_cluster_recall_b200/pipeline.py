@@ -111,6 +111,15 @@ class ClusterRecall:
         return self.out
 
     def step(self, q, K, V) -> torch.Tensor:
+        """One decode step: selection then sparse attention, as one fused
+        launch (ckv_select_decode) when the shape allows it."""
+        if self.G in (1, 2, 4):
+            ckv.ckv_select_decode(q, self.centroids_lp, self.n_clusters, self.C_cap,
+                                  self.offsets, self.perm, self.perm_cap, self.B, self.sel_idx,
+                                  self.sel_cnt, K, V, K.stride(0), self.kv_rows, self.S,
+                                  self.tail_begin, self.tail_end, self.max_tail, self.scale,
+                                  self.out, P=self.P, G=self.G, d=self.d, stream=self.stream)
+            return self.out
         self.select(q)
         return self.decode(q, K, V)
 
