@@ -81,7 +81,7 @@ cudaError_t smem_optin(K kernel, size_t bytes, int slot) {
 
 // slots for smem_optin (one per kernel instantiation that may exceed 48 KB)
 enum { SLOT_ASSIGN_F32 = 0, SLOT_ASSIGN_BF16, SLOT_HIST, SLOT_SCATTER, SLOT_RANK, SLOT_ASSIGN_TC,
-       SLOT_SD_BASE /* + 6 fused select-decode instantiations */ };
+       SLOT_SD_BASE /* + 10 fused select-decode instantiations */ };
 
 bool valid_dtype(ckv_dtype dt) { return dt == CKV_F32 || dt == CKV_BF16; }
 
@@ -448,6 +448,9 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
         return fail(CKV_ERR_UNSUPPORTED, "fused step supports up to %d attended rows per problem",
                     sd::NC_MAX * sd::POS_MAX);
     const size_t smem = sd::layout(C_cap, G, chunk, nc).total;
+    // rows in flight per half-warp: one batch for the CTA's rows when the
+    // registers allow it (16 half-warps per CTA)
+    const int U = (G == 4) ? 6 : (chunk <= 16 * 4 ? 4 : 9);
     sd::Args a;
     a.q = q;
     a.lp = centroids_lp;
@@ -482,19 +485,19 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaSuccess;
-#define CKV_SD(T, GG)                                                                     \
-    do {                                                                                  \
-        e = smem_optin(sd::k_select_decode<T, GG>, smem, SLOT_SD_BASE + (sizeof(T) == 2) * 3 + (GG == 1 ? 0 : GG == 2 ? 1 : 2)); \
-        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sd::k_select_decode<T, GG>, a); \
+#define CKV_SD(T, GG, UU, SLOT)                                                            \
+    do {                                                                                   \
+        e = smem_optin(sd::k_select_decode<T, GG, UU>, smem, SLOT_SD_BASE + (SLOT));       \
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sd::k_select_decode<T, GG, UU>, a); \
     } while (0)
     if (dt == CKV_BF16) {
-        if (G == 1) CKV_SD(bf16, 1);
-        else if (G == 2) CKV_SD(bf16, 2);
-        else CKV_SD(bf16, 4);
+        if (G == 4) CKV_SD(bf16, 4, 6, 0);
+        else if (G == 2) { if (U == 4) CKV_SD(bf16, 2, 4, 1); else CKV_SD(bf16, 2, 9, 2); }
+        else { if (U == 4) CKV_SD(bf16, 1, 4, 3); else CKV_SD(bf16, 1, 9, 4); }
     } else {
-        if (G == 1) CKV_SD(float, 1);
-        else if (G == 2) CKV_SD(float, 2);
-        else CKV_SD(float, 4);
+        if (G == 4) CKV_SD(float, 4, 6, 5);
+        else if (G == 2) { if (U == 4) CKV_SD(float, 2, 4, 6); else CKV_SD(float, 2, 9, 7); }
+        else { if (U == 4) CKV_SD(float, 1, 4, 8); else CKV_SD(float, 1, 9, 9); }
     }
 #undef CKV_SD
     if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "k_select_decode: %s", cudaGetErrorString(e));

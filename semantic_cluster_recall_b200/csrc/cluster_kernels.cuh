@@ -14,9 +14,53 @@
 
 namespace ckv {
 
+// Round a double to bf16 (round to nearest, ties to even) in one step, from
+// the bit pattern: 8 significant bits are kept and the 45 dropped mantissa
+// bits decide the rounding. Values below the fp32 normal range take the
+// fp32 path (two roundings), which no centroid of unit-scale keys reaches.
+__device__ __forceinline__ uint16_t bf16_bits_rn(double x) {
+    const unsigned long long b = (unsigned long long)__double_as_longlong(x);
+    const unsigned sign = (unsigned)(b >> 63) << 15;
+    const int e = (int)((b >> 52) & 0x7ff) - 1023;
+    if (x != x) return (uint16_t)(sign | 0x7fc0u);
+    if (e > 127) return (uint16_t)(sign | 0x7f80u);
+    if (e < -126) return __bfloat16_as_ushort(__float2bfloat16_rn((float)x));
+    const unsigned long long m = b & ((1ull << 52) - 1);
+    unsigned keep = (unsigned)(m >> 45);              // 7 stored mantissa bits
+    const unsigned long long rem = m & ((1ull << 45) - 1);
+    const unsigned long long halfway = 1ull << 44;
+    unsigned v = ((unsigned)(e + 127) << 7) | keep;   // exponent and mantissa
+    if (rem > halfway || (rem == halfway && (keep & 1u))) v += 1;  // may carry into the exponent
+    if (v >= 0x7f80u) v = 0x7f80u;                    // rounded past the largest finite
+    return (uint16_t)(sign | v);
+}
+
+template <typename T>
+__device__ __forceinline__ void store4_rn(T *p, const double (&v)[4]);
+
+template <>
+__device__ __forceinline__ void store4_rn<float>(float *p, const double (&v)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4((float)v[0], (float)v[1], (float)v[2], (float)v[3]);
+}
+
+template <>
+__device__ __forceinline__ void store4_rn<bf16>(bf16 *p, const double (&v)[4]) {
+    uint2 u;
+    u.x = (uint32_t)bf16_bits_rn(v[0]) | ((uint32_t)bf16_bits_rn(v[1]) << 16);
+    u.y = (uint32_t)bf16_bits_rn(v[2]) | ((uint32_t)bf16_bits_rn(v[3]) << 16);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+
 // ---------------------------------------------------------------------------
 // a1 seeding: centroid c starts at the key of position tok_begin + c*floor(n/C).
-// One warp per centroid; lane l owns channels 4l..4l+3.
+// One warp per centroid; lane l owns channels 4l..4l+3. The unit copy is
+// normalised in double and rounded to the storage type once.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -28,17 +72,19 @@ k_init(const T *__restrict__ keys, int64_t pstride, int tok_begin, int n, int C,
     if (c >= C) return;
     const int stride = n / C;
     const T *row = keys + (int64_t)p * pstride + (int64_t)(tok_begin + c * stride) * D;
-    float4 v = load4(row + lane * 4);
-    float ss = warp_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w);
+    const float4 v = load4(row + lane * 4);
+    const double mu[4] = {v.x, v.y, v.z, v.w};  // exact
+    const double ss = warp_sum_d(mu[0] * mu[0] + mu[1] * mu[1] + mu[2] * mu[2] + mu[3] * mu[3]);
     const size_t o = ((size_t)p * C_cap + cbase + c) * D + lane * 4;
     store4(cent + o, v);
     store4(lp + o, v);
-    float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (ss > 0.f) {
-        float nrm = sqrtf(ss);
-        h = make_float4(v.x / nrm, v.y / nrm, v.z / nrm, v.w / nrm);
+    double h[4] = {0.0, 0.0, 0.0, 0.0};
+    if (ss > 0.0) {
+        const double nrm = sqrt(ss);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) h[t] = mu[t] / nrm;
     }
-    store4(hat + o, h);
+    store4_rn(hat + o, h);
 }
 
 // ---------------------------------------------------------------------------
@@ -292,32 +338,44 @@ k_index_scatter(const int32_t *__restrict__ labels, int perm_base, int perm_cap,
 
 // ---------------------------------------------------------------------------
 // a3 centroid update: one warp per cluster gathers its member rows through
-// perm. A 16-lane half-warp owns one row at a time (16 bytes per lane for
-// bf16, i.e. a whole 256-byte row per half-warp) and keeps 8 rows in flight;
-// the two halves take alternate rows and are added at the end. Sums are fp32,
-// in a fixed order (deterministic, no atomics); then the mean, its norm, and
-// the two rounded copies.
+// perm; lane l owns channels 4l..4l+3 (one 256-byte bf16 row per warp load)
+// and keeps UPD_ROWS rows in flight. Each channel is summed in double, one
+// row at a time in perm order (ascending position), so the sum, the mean,
+// and the rounded copies do not depend on the launch shape. Deterministic,
+// no atomics.
 // ---------------------------------------------------------------------------
-constexpr int UPD_ROWS = 8;  // rows in flight per half-warp
+constexpr int UPD_ROWS = 16;  // rows in flight per warp
 
+// Raw bits of 4 consecutive elements (loaded first, converted later, so all
+// loads of a batch are in flight together).
 template <typename T>
-__device__ __forceinline__ void store8(T *p, const float (&v)[8]);
+struct Raw4;
 
 template <>
-__device__ __forceinline__ void store8<float>(float *p, const float (&v)[8]) {
-    reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
+struct Raw4<bf16> {
+    uint2 u;
+    __device__ __forceinline__ void load(const bf16 *p) { u = __ldg(reinterpret_cast<const uint2 *>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint2(0, 0); }
+    __device__ __forceinline__ void add_to(double (&acc)[4]) const {
+        acc[0] += (double)__uint_as_float(u.x << 16);
+        acc[1] += (double)__uint_as_float(u.x & 0xffff0000u);
+        acc[2] += (double)__uint_as_float(u.y << 16);
+        acc[3] += (double)__uint_as_float(u.y & 0xffff0000u);
+    }
+};
 
 template <>
-__device__ __forceinline__ void store8<bf16>(bf16 *p, const float (&v)[8]) {
-    uint4 u;
-    u.x = pack_bf16x2(v[0], v[1]);
-    u.y = pack_bf16x2(v[2], v[3]);
-    u.z = pack_bf16x2(v[4], v[5]);
-    u.w = pack_bf16x2(v[6], v[7]);
-    *reinterpret_cast<uint4 *>(p) = u;
-}
+struct Raw4<float> {
+    float4 f;
+    __device__ __forceinline__ void load(const float *p) { f = __ldg(reinterpret_cast<const float4 *>(p)); }
+    __device__ __forceinline__ void zero() { f = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void add_to(double (&acc)[4]) const {
+        acc[0] += (double)f.x;
+        acc[1] += (double)f.y;
+        acc[2] += (double)f.z;
+        acc[3] += (double)f.w;
+    }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -326,7 +384,6 @@ k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end
          const int32_t *__restrict__ perm, int perm_cap, float *__restrict__ cent,
          T *__restrict__ hat, T *__restrict__ lp, int32_t *__restrict__ sizes) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half = lane >> 4, hl = lane & 15;
     const int c = blockIdx.x * 8 + warp;
     const int p = blockIdx.y;
     if (c >= C) return;
@@ -340,61 +397,44 @@ k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end
         }
         return;
     }
-    const T *kb = keys + (int64_t)p * pstride + hl * 8;
+    const T *kb = keys + (int64_t)p * pstride + lane * 4;
     const int32_t *pp = perm + (size_t)p * perm_cap;
-    float acc[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
     for (int j0 = o0; j0 < o1; j0 += 32) {
         const int cnt = min(32, o1 - j0);
         const int pos = lane < cnt ? pp[j0 + lane] : -1;
-        for (int k = 0; k < cnt; k += 2 * UPD_ROWS) {
-            Row8<T> r[UPD_ROWS];
+        for (int k = 0; k < cnt; k += UPD_ROWS) {
+            Raw4<T> r[UPD_ROWS];
 #pragma unroll
             for (int u = 0; u < UPD_ROWS; ++u) {
-                const int kk = k + 2 * u + half;  // < 32 always
+                const int kk = k + u;  // < 32 always
                 const int ps = __shfl_sync(FULL, pos, kk & 31);
                 r[u].zero();
                 if (kk < cnt) {
                     if (ps >= tok_begin && ps < tok_end) r[u].load(kb + (int64_t)ps * D);
-                    else if (hl == 0) dev_flag(CKV_DEVERR_PERM);
+                    else if (lane == 0) dev_flag(CKV_DEVERR_PERM);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < UPD_ROWS; ++u) {
-                float f[8];
-                r[u].to_float(f);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) acc[t] += f[t];
-            }
+            for (int u = 0; u < UPD_ROWS; ++u) r[u].add_to(acc);  // perm order; +0 is exact
         }
     }
-#pragma unroll
-    for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(FULL, acc[t], 16);
     const int n = o1 - o0;
     if (lane == 0) *sz = n;
     if (n == 0) return;
-    const float fn = (float)n;
-    float mu[8];
-    float ss = 0.f;
+    double mu[4];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-        mu[t] = acc[t] / fn;
-        ss = fmaf(mu[t], mu[t], ss);
-    }
+    for (int t = 0; t < 4; ++t) mu[t] = acc[t] / (double)n;
+    const double ss = warp_sum_d(mu[0] * mu[0] + mu[1] * mu[1] + mu[2] * mu[2] + mu[3] * mu[3]);
+    if (!(ss > 0.0)) return;
+    const double nrm = sqrt(ss);
+    double h[4];
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
-    if (!(ss > 0.f)) return;
-    if (half == 0) {
-        const float nrm = sqrtf(ss);
-        float h[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) h[t] = mu[t] / nrm;
-        const size_t o = ((size_t)p * C_cap + cbase + c) * D + hl * 8;
-        store8<float>(cent + o, mu);
-        store8<T>(lp + o, mu);
-        store8<T>(hat + o, h);
-    }
+    for (int t = 0; t < 4; ++t) h[t] = mu[t] / nrm;
+    const size_t o = ((size_t)p * C_cap + cbase + c) * D + lane * 4;
+    store4_rn<float>(cent + o, mu);
+    store4_rn<T>(lp + o, mu);
+    store4_rn<T>(hat + o, h);
 }
 
 }  // namespace ckv

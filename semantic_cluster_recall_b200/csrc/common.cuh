@@ -76,6 +76,9 @@ struct Row8<bf16> {
     __device__ __forceinline__ void load(const bf16 *p) {
         u = __ldg(reinterpret_cast<const uint4 *>(p));
     }
+    __device__ __forceinline__ void load_shared(const bf16 *p) {
+        u = *reinterpret_cast<const uint4 *>(p);
+    }
     __device__ __forceinline__ void zero() { u = make_uint4(0, 0, 0, 0); }
     __device__ __forceinline__ void to_float(float (&f)[8]) const { unpack8(u, f); }
 };
@@ -86,6 +89,10 @@ struct Row8<float> {
     __device__ __forceinline__ void load(const float *p) {
         a = __ldg(reinterpret_cast<const float4 *>(p));
         b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    }
+    __device__ __forceinline__ void load_shared(const float *p) {
+        a = reinterpret_cast<const float4 *>(p)[0];
+        b = reinterpret_cast<const float4 *>(p)[1];
     }
     __device__ __forceinline__ void zero() {
         a = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -9,8 +9,9 @@
 //              fixed fp32 order of k_score and writes the 64-bit rank key
 //              (descending score, ascending id) into every CTA's key table
 //   -- cluster barrier
-//   2. rank    CTA r ranks clusters c = r (mod NC) by counting smaller keys
-//              and writes (order[rank] = c, size[rank] = n_c) into every CTA
+//   2. rank    CTA r ranks clusters c = r (mod NC), one warp per cluster,
+//              the 32 lanes counting smaller keys, and writes
+//              (order[rank] = c, size[rank] = n_c) into every CTA
 //   -- cluster barrier
 //   3. fill    every CTA prefix-sums the sizes in rank order (redundantly, no
 //              leader round trip); sel_cnt = min(budget, total)
@@ -19,7 +20,9 @@
 //              binary search and its position through offsets/perm; the
 //              positions go to shared memory and to sel_idx (ABI output)
 //   5. attend  split-K online softmax over the CTA's rows (half-warp per
-//              256-byte row, 8 rows in flight), merged inside the CTA
+//              256-byte row, U rows in flight per half-warp, U chosen so a
+//              CTA's rows arrive in one batch at the usual shapes), merged
+//              inside the CTA
 //   -- partial (m, l, o) pushed into the leader CTA's shared memory
 //   -- cluster barrier
 //   6. combine the leader merges the NC partials and writes out
@@ -41,7 +44,6 @@ namespace cg = cooperative_groups;
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
 constexpr int HALVES = THREADS / 16;   // row streams
-constexpr int U = 8;                   // rows in flight per half-warp
 constexpr int NC_MAX = 8;              // CTAs per problem (portable cluster size)
 constexpr int POS_MAX = 4096;          // attended rows per CTA
 
@@ -70,7 +72,7 @@ struct Args {
 
 // dynamic shared memory layout (bytes), sized by C_cap, G and chunk
 struct Layout {
-    size_t keys, order, size, start, pos, mo, ml, part, total;
+    size_t keys, order, size, start, offs, pos, mo, ml, part, total;
 };
 
 __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -82,6 +84,7 @@ __host__ __device__ inline Layout layout(int C_cap, int G, int chunk, int nc) {
     L.order = o;  o += al16((size_t)C_cap * 4);
     L.size = o;   o += al16((size_t)C_cap * 4);
     L.start = o;  o += al16((size_t)(C_cap + 1) * 4);
+    L.offs = o;   o += al16((size_t)(C_cap + 1) * 4);     // the problem's offsets row
     L.pos = o;    o += al16((size_t)chunk * 4);
     L.mo = o;     o += al16((size_t)HALVES * D * 4);          // per-g merge of the row streams
     L.ml = o;     o += al16((size_t)HALVES * 2 * 4);
@@ -90,7 +93,7 @@ __host__ __device__ inline Layout layout(int C_cap, int G, int chunk, int nc) {
     return L;
 }
 
-template <typename T, int G>
+template <typename T, int G, int U>
 __global__ void __launch_bounds__(THREADS)
 k_select_decode(const Args a) {
     cg::cluster_group cl = cg::this_cluster();
@@ -104,6 +107,7 @@ k_select_decode(const Args a) {
     int32_t *order = reinterpret_cast<int32_t *>(smem + LY.order);
     int32_t *rsz = reinterpret_cast<int32_t *>(smem + LY.size);
     int32_t *start = reinterpret_cast<int32_t *>(smem + LY.start);
+    int32_t *off_s = reinterpret_cast<int32_t *>(smem + LY.offs);
     int32_t *pos_s = reinterpret_cast<int32_t *>(smem + LY.pos);
     float *mo = reinterpret_cast<float *>(smem + LY.mo);
     float *mml = reinterpret_cast<float *>(smem + LY.ml);
@@ -115,6 +119,8 @@ k_select_decode(const Args a) {
     const int32_t *pp = a.perm + (size_t)p * a.perm_cap;
     const T *qp = reinterpret_cast<const T *>(a.q) + (size_t)p * G * D;
 
+    // the problem's offsets row, needed by ranking and by position lookup
+    for (int i = tid; i <= nC; i += THREADS) off_s[i] = off[i];
     cl.sync();  // every CTA of the cluster is running before any DSMEM access
 
     // ---- 1. score (fixed fp32 order), keys broadcast to every CTA ----
@@ -123,57 +129,61 @@ k_select_decode(const Args a) {
 #pragma unroll
         for (int g = 0; g < G; ++g) qv[g] = load4(qp + g * D + lane * 4);
         const T *lpp = reinterpret_cast<const T *>(a.lp) + (size_t)p * a.C_cap * D + lane * 4;
-        for (int c = rank * WARPS + warp; c < nC; c += nc * WARPS) {
-            const float4 m = load4(lpp + (size_t)c * D);
-            float tot = 0.f;
+        const int cstride = nc * WARPS;
+        constexpr int SB = 8;  // centroid rows in flight per warp
+        for (int cb = rank * WARPS + warp; cb < nC; cb += cstride * SB) {
+            float4 mrow[SB];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float s = 0.f;
-                s = fmaf(qv[g].x, m.x, s);
-                s = fmaf(qv[g].y, m.y, s);
-                s = fmaf(qv[g].z, m.z, s);
-                s = fmaf(qv[g].w, m.w, s);
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) s = s + __shfl_xor_sync(FULL, s, o);
-                tot = (g == 0) ? s : tot + s;
+            for (int u = 0; u < SB; ++u) {
+                const int c = cb + u * cstride;
+                mrow[u] = c < nC ? load4(lpp + (size_t)c * D) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            const uint64_t key = ((uint64_t)(~ordered_bits(tot)) << 32) | (uint32_t)c;
-            if (lane < nc) *cl.map_shared_rank(&keys[c], lane) = key;
+#pragma unroll
+            for (int u = 0; u < SB; ++u) {
+                const int c = cb + u * cstride;
+                if (c >= nC) break;  // warp-uniform
+                float tot = 0.f;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float sc = 0.f;
+                    sc = fmaf(qv[g].x, mrow[u].x, sc);
+                    sc = fmaf(qv[g].y, mrow[u].y, sc);
+                    sc = fmaf(qv[g].z, mrow[u].z, sc);
+                    sc = fmaf(qv[g].w, mrow[u].w, sc);
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) sc = sc + __shfl_xor_sync(FULL, sc, o);
+                    tot = (g == 0) ? sc : tot + sc;
+                }
+                const uint64_t key = ((uint64_t)(~ordered_bits(tot)) << 32) | (uint32_t)c;
+                if (lane < nc) *cl.map_shared_rank(&keys[c], lane) = key;
+            }
         }
     }
     cl.sync();
 
-    // ---- 2. rank own clusters (c = rank mod nc), broadcast order and sizes ----
-    {
-        const int nown = nC > rank ? (nC - rank + nc - 1) / nc : 0;
-        // threads per cluster: a power of two so the partial counts add by shuffles
-        int tpc = 32;
-        while (tpc > 1 && tpc * nown > THREADS) tpc >>= 1;
-        const int slot = tid / tpc, sub = tid % tpc;
-        const int per_pass = THREADS / tpc;
-        for (int base = 0; base < nown; base += per_pass) {
-            const int i = base + slot;
-            const bool mine = i < nown;
-            const int c = rank + i * nc;
-            int cnt = 0;
-            if (mine) {
-                const uint64_t kc = keys[c];
-                for (int k = sub; k < nC; k += tpc) cnt += keys[k] < kc;
-            }
-            for (int o = tpc >> 1; o >= 1; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
-            if (mine) {
-                int sz = 0;
-                const int o0 = off[c], o1 = off[c + 1];
-                if (o0 < 0 || o1 < o0 || o1 > a.perm_cap) {
-                    if (sub == 0) dev_flag(CKV_DEVERR_OFFSETS);
-                } else {
-                    sz = o1 - o0;
-                }
-                for (int r = sub; r < nc; r += tpc) {  // every CTA gets (order, size)
-                    *cl.map_shared_rank(&order[cnt], r) = c;
-                    *cl.map_shared_rank(&rsz[cnt], r) = sz;
-                }
-            }
+    // ---- 2. rank own clusters (c = rank mod nc): one warp per cluster ----
+    for (int c = rank + warp * nc; c < nC; c += WARPS * nc) {  // warp-uniform
+        const uint64_t kc = keys[c];
+        int n0 = 0, n1 = 0, n2 = 0, n3 = 0;  // independent partial counts
+        int k = lane;
+        for (; k + 96 < nC; k += 128) {
+            n0 += keys[k] < kc;
+            n1 += keys[k + 32] < kc;
+            n2 += keys[k + 64] < kc;
+            n3 += keys[k + 96] < kc;
+        }
+        for (; k < nC; k += 32) n0 += keys[k] < kc;
+        const int r = __reduce_add_sync(FULL, n0 + n1 + n2 + n3);
+        int sz = 0;
+        const int o0 = off_s[c], o1 = off_s[c + 1];
+        if (o0 < 0 || o1 < o0 || o1 > a.perm_cap) {
+            if (lane == 0) dev_flag(CKV_DEVERR_OFFSETS);
+        } else {
+            sz = o1 - o0;
+        }
+        if (lane < nc) {  // every CTA gets (order, size)
+            *cl.map_shared_rank(&order[r], lane) = c;
+            *cl.map_shared_rank(&rsz[r], lane) = sz;
         }
     }
     cl.sync();
@@ -226,7 +236,7 @@ k_select_decode(const Args a) {
                 else hi = mid - 1;
             }
             const int c = order[lo];
-            const int slot = off[c] + (k - start[lo]);
+            const int slot = off_s[c] + (k - start[lo]);
             row = (slot >= 0 && slot < a.perm_cap) ? pp[slot] : -1;
             a.sel_idx[(size_t)p * a.B + k] = row;
         } else {
@@ -280,38 +290,54 @@ k_select_decode(const Args a) {
                 vr[u].zero();
             }
         }
-        float kf[U][8];
+        float lg[G][U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) kr[u].to_float(kf[u]);
+        for (int u = 0; u < U; ++u) {
+            float kf[8];
+            kr[u].to_float(kf);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float lg[U];
-            float mx = m[g];
+            for (int g = 0; g < G; ++g) {
+                float sc = 0.f;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) sc = fmaf(qf[g][t], kf[t], sc);
+                lg[g][u] = sc;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                float s = 0.f;
 #pragma unroll
-                for (int t = 0; t < 8; ++t) s = fmaf(qf[g][t], kf[u][t], s);
-#pragma unroll
-                for (int w = 8; w >= 1; w >>= 1) s += __shfl_xor_sync(FULL, s, w);
-                lg[u] = row[u] >= 0 ? s : -INFINITY;
-                mx = fmaxf(mx, lg[u]);
+                for (int w = 8; w >= 1; w >>= 1) lg[g][u] += __shfl_xor_sync(FULL, lg[g][u], w);
+                if (row[u] < 0) lg[g][u] = -INFINITY;
             }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float mx = m[g];
+#pragma unroll
+            for (int u = 0; u < U; ++u) mx = fmaxf(mx, lg[g][u]);
             if (mx != -INFINITY) {
                 const float corr = exp2f(m[g] - mx);
                 l[g] *= corr;
 #pragma unroll
                 for (int t = 0; t < 8; ++t) o[g][t] *= corr;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const float pu = exp2f(lg[u] - mx);
-                    l[g] += pu;
-                    float vf[8];
-                    vr[u].to_float(vf);
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) o[g][t] = fmaf(pu, vf[t], o[g][t]);
-                }
                 m[g] = mx;
+#pragma unroll
+                for (int u = 0; u < U; ++u) lg[g][u] = exp2f(lg[g][u] - mx);
+            } else {
+#pragma unroll
+                for (int u = 0; u < U; ++u) lg[g][u] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float vf[8];
+            vr[u].to_float(vf);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                l[g] += lg[g][u];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) o[g][t] = fmaf(lg[g][u], vf[t], o[g][t]);
             }
         }
     }
