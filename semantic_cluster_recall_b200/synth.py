@@ -187,6 +187,19 @@ def make_queries(w: Workload, step: int = 0, device="cpu",
     return out
 
 
+def directions_all(w: Workload, device) -> torch.Tensor:
+    """Mixture directions of every problem, [P, M, d] (fp32)."""
+    return torch.stack([directions(w, p, device) for p in range(w.P)])
+
+
+def make_queries_batched(w: Workload, dirs: torch.Tensor, step: int) -> torch.Tensor:
+    """Decode queries [P, G, d] for step `step` drawn for all problems at once
+    from one generator stream per step (for long decode loops over many
+    problems; a different stream than make_queries)."""
+    g = _gen(dirs.device, w.seed, 6_000_000 + step)
+    return mixture_rows(dirs, w.G, w.sigma, g, scale=w.q_scale).to(w.torch_dtype)
+
+
 def random_labels(P: int, n: int, C: int, seed: int, device="cpu",
                   skew: float = 0.0) -> torch.Tensor:
     """Seeded cluster labels [P, n] int32 in [0, C), for stage-level tests.
@@ -218,4 +231,5 @@ def ceil_div(a: int, b: int) -> int:
 
 
 __all__ = ["Workload", "WORKLOADS", "WORKLOAD_ORDER", "make_kv", "make_queries",
-           "random_labels", "mixture_rows", "directions", "describe", "ceil_div"]
+           "make_queries_batched", "directions_all", "random_labels", "mixture_rows",
+           "directions", "describe", "ceil_div"]
