@@ -32,7 +32,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # CKV_ORACLE_LIB points the pins at another build of the oracle (the
+        # mutation tests use it to show that planted mistakes are caught)
+        path = os.environ.get("CKV_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         f32p = np.ctypeslib.ndpointer(np.float32, flags="C")
         f64p = np.ctypeslib.ndpointer(np.float64, flags="C")

@@ -15,12 +15,12 @@ FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-sh
          "-Wall", "-Wextra"]
 
 
-def build(force: bool = False, out: str = LIB, defines=()) -> str:
+def build(force: bool = False, out: str = LIB, defines=(), src: str = SRC) -> str:
     """Compile the oracle if the library is missing or older than its source."""
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(SRC):
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
         return out
     tmp = out + ".tmp%d" % os.getpid()
-    cmd = ["gcc", *FLAGS, *["-D" + x for x in defines], SRC, "-o", tmp, "-lm"]
+    cmd = ["gcc", *FLAGS, *["-D" + x for x in defines], src, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
     return out
