@@ -82,26 +82,37 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, interval_ms: int = 20):
         self.index = index
+        self.interval_ms = interval_ms
         self.proc = None
         self.lines = []
+        self.first = threading.Event()
+        self.window = None  # (first, last) sample index inside the timed region
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            self.first.wait(timeout=5.0)  # sampling is running before the timed region
         except OSError:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self._w0 = len(self.lines)
+
+    def mark_end(self):
+        self.window = (getattr(self, "_w0", 0), len(self.lines))
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+            self.first.set()
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -115,7 +126,11 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.window and self.window[1] > self.window[0]:
+            # samples taken while the timed steps ran, plus the one just before
+            lines = self.lines[max(0, self.window[0] - 1):self.window[1] + 1]
+        for ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -232,6 +247,59 @@ def time_decode_steps(step: Step, n: int):
     return times
 
 
+def decode_32layer(dev, stream, n_steps: int = 20) -> dict:
+    """Decode steps of the full 32-layer model (batch 4, 32 KV heads per
+    layer: 4096 problems at 32k context): one prefill clustering of all of
+    them, then graph-replayed fused decode steps over all 4096 problems."""
+    w = synth.WORKLOADS["llama2_32layer_decode"]
+    pk = peaks()
+    K, V = synth.make_kv(w, device=dev, rows=w.L)
+    dirs = synth.directions_all(w, dev)
+    q = synth.make_queries_batched(w, dirs, 1)
+    del dirs
+    st = ClusterRecall(w.P, w.G, w.d, w.torch_dtype, w.L, w.S, w.B, w.C, w.N, w.W, dev,
+                       stream=stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    st.prefill(K, w.L, w.W, w.C, w.T)  # warm-up
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    st.prefill(K, w.L, w.W, w.C, w.T)
+    b.record(stream)
+    b.synchronize()
+    t_cluster = a.elapsed_time(b) * 1e-3
+    st.step(q, K, V)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        st.step(q, K, V)
+    times = []
+    for _ in range(n_steps):
+        flush.random_(0, 255)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    del g
+    t = statistics.median(times)
+    byts = decode_bytes(w.replace(tail_cap=0))
+    res = {"workload": w.name, "P": w.P, "steps_per_s": 1.0 / t, "us_per_step": t * 1e6,
+           "bytes_per_step": byts,
+           "roofline": {"bound": "hbm", "achieved": byts / t / 1e9, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": byts / t / 1e9 / pk["hbm_gbs"],
+                        "peak_source": pk["source"] + " copy"},
+           "prefill_clustering": {"keys_per_s": w.P * w.N / t_cluster,
+                                  "ms": t_cluster * 1e3, "keys": w.P * w.N},
+           "launch": "fused select + sparse decode, CUDA graph replay, L2 flushed"}
+    del K, V, st, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def e2e_measure(w: synth.Workload, dev, stream, steps: int):
     """End to end through the public calls: pinned host K/V/q -> device, one
     ckv_cluster + ckv_select + ckv_sparse_decode, outputs -> pinned host."""
@@ -323,12 +391,14 @@ def run_ours(args):
         barrier(world)
         torch.cuda.synchronize()
         with ClockSampler(local) as clk:
+            clk.mark_start()
             for k in range(args.steps):
                 step.flush_l2()
                 ev_steps[k][0].record(stream)
                 step.run(ev_assign[k], ev_dec[k])
                 ev_steps[k][1].record(stream)
             torch.cuda.synchronize()
+            clk.mark_end()
         barrier(world)
         step_s = [a.elapsed_time(b) * 1e-3 for a, b in ev_steps]
         assign_s = [a.elapsed_time(b) * 1e-3 for row in ev_assign for a, b in row]
@@ -338,6 +408,14 @@ def run_ours(args):
         err = ckv.ckv_device_error()
         e2e_s, h2d, d2h = e2e_measure(w, dev, stream, max(2, min(args.steps, 3)))
         e2e_s = reduce_max(e2e_s, world, dev)
+        del step
+        torch.cuda.empty_cache()
+        dec32 = None
+        if world == 1 and not args.no_32layer:
+            try:
+                dec32 = decode_32layer(dev, stream)
+            except Exception as ex:  # reported, never fatal for the main line
+                dec32 = {"error": f"{type(ex).__name__}: {ex}"[:300]}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -351,7 +429,7 @@ def run_ours(args):
     achieved_tf = flops / t_assign / 1e12
     dec_bytes = decode_bytes(w)
     t_dec = statistics.median(dec_steps)
-    launches = step.launches_per_step * args.steps
+    launches = (1 + w.T * 5 + (1 if w.G in (1, 2, 4) else 4)) * args.steps
     line = {
         "metric": METRIC,
         "value": value,
@@ -387,6 +465,7 @@ def run_ours(args):
                    "launch": "fused select + sparse decode (one cluster launch), CUDA graph replay"},
         "e2e": {"value": world * keys / e2e_s, "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
+        "decode_32layer": dec32,
         "gpu_launches": launches,
         "device_error_flags": err,
     }
@@ -480,11 +559,13 @@ def run_only(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-32layer", action="store_true",
+                    help="skip the 32-layer (4096-problem) decode measurement")
     ap.add_argument("--only", choices=["assign", "index", "update", "select", "decode", "step"],
                     help="run one stage --launches times (profiler captures); prints no metric")
     ap.add_argument("--launches", type=int, default=3)
