@@ -275,3 +275,50 @@ def test_decode_peaked_softmax_and_no_rows(cuda_device):
     _decode_case(cuda_device, torch.bfloat16, P=3, G=2, L=3000, S=0, sel_counts=[2048, 5, 0],
                  tails=[(2900, 3000), (2990, 3000), (2999, 2999)], budget=2048, q_scale=12.0,
                  seed=7)
+
+
+# ---- edge cases ----------------------------------------------------------------
+
+def test_assign_every_token_its_own_cluster_and_zero_keys(cuda_device):
+    # C = n: seeds are the keys themselves, so each key's best centroid is its
+    # own (by a wide margin); zero keys score 0 against every centroid and go
+    # to the lowest index on both sides.
+    dev = cuda_device
+    w = small_workload(torch.bfloat16, P=2, L=1100, S=4, W=96, C=1000, M=64)
+    K, V = synth.make_kv(w)
+    K[:, 100:103] = 0  # three zero keys inside the clustered region
+    Kh = f32np(K)
+    tb, te = w.S, w.L - w.W
+    n = te - tb
+    assert n == w.C
+    Kd = K.to(dev)
+    hat_np = np.zeros((w.P, w.C, 128), np.float32)
+    for p in range(w.P):
+        hat_np[p] = oracle.init(Kh[p, tb:te], w.C, "bf16")[1]
+    labels = torch.full((w.P, n), -1, dtype=torch.int32, device=dev)
+    ckv.ckv_assign(Kd, Kd.stride(0), tb, te, to_dev(hat_np, torch.bfloat16, dev), w.C, 0, w.C,
+                   labels, 0, n)
+    torch.cuda.synchronize()
+    lab = labels.cpu().numpy()
+    for p in range(w.P):
+        ref, gap = oracle.assign(Kh[p, tb:te], hat_np[p].astype(np.float64))
+        bad = (lab[p] != ref) & (gap >= GAP_EXEMPT)
+        assert not bad.any()
+        zero = np.all(Kh[p, tb:te] == 0, axis=1)
+        assert zero.sum() == 3 and np.all(lab[p][zero] == 0) and np.all(ref[zero] == 0)
+        nz = np.where(~zero)[0]
+        # nonzero keys pick themselves unless a parallel duplicate exists (none here)
+        assert np.mean(lab[p][nz] == nz) > 0.999
+    assert ckv.ckv_device_error() == 0
+
+
+def test_select_max_clusters(cuda_device):
+    # C_cap = C + 5 = 4096, the largest supported
+    _select_case(cuda_device, torch.bfloat16, P=2, G=1, C=4091, n=40000, budget=2048, seed=21)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_select_and_decode_eight_query_heads(cuda_device, dtype):
+    _select_case(cuda_device, dtype, P=3, G=8, C=300, n=3000, budget=512, seed=8)
+    _decode_case(cuda_device, dtype, P=3, G=8, L=4000, S=16, sel_counts=[512, 100, 0],
+                 tails=[(3936, 4000), (3900, 4000), (3990, 3990)], budget=512, seed=9)
