@@ -81,7 +81,7 @@ cudaError_t smem_optin(K kernel, size_t bytes, int slot) {
 
 // slots for smem_optin (one per kernel instantiation that may exceed 48 KB)
 enum { SLOT_ASSIGN_F32 = 0, SLOT_ASSIGN_BF16, SLOT_HIST, SLOT_SCATTER, SLOT_RANK, SLOT_ASSIGN_TC,
-       SLOT_SD_BASE /* + 10 fused select-decode instantiations */ };
+       SLOT_SD_BASE /* + 12 fused select-decode instantiations */ };
 
 bool valid_dtype(ckv_dtype dt) { return dt == CKV_F32 || dt == CKV_BF16; }
 
@@ -449,8 +449,10 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
                     sd::NC_MAX * sd::POS_MAX);
     const size_t smem = sd::layout(C_cap, G, chunk, nc).total;
     // rows in flight per half-warp: one batch for the CTA's rows when the
-    // registers allow it (16 half-warps per CTA)
-    const int U = (G == 4) ? 6 : (chunk <= 16 * 4 ? 4 : 9);
+    // registers allow it (16 half-warps per CTA); when a problem is a single
+    // CTA (many problems), fewer rows and registers, so that 4 CTAs share an
+    // SM and their selection phases overlap each other's gathers
+    const int U = (G == 4) ? (nc == 1 ? 2 : 6) : ((chunk <= 16 * 4 || nc == 1) ? 4 : 9);
     sd::Args a;
     a.q = q;
     a.lp = centroids_lp;
@@ -491,11 +493,11 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
         if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sd::k_select_decode<T, GG, UU>, a); \
     } while (0)
     if (dt == CKV_BF16) {
-        if (G == 4) CKV_SD(bf16, 4, 6, 0);
+        if (G == 4) { if (U == 2) CKV_SD(bf16, 4, 2, 10); else CKV_SD(bf16, 4, 6, 0); }
         else if (G == 2) { if (U == 4) CKV_SD(bf16, 2, 4, 1); else CKV_SD(bf16, 2, 9, 2); }
         else { if (U == 4) CKV_SD(bf16, 1, 4, 3); else CKV_SD(bf16, 1, 9, 4); }
     } else {
-        if (G == 4) CKV_SD(float, 4, 6, 5);
+        if (G == 4) { if (U == 2) CKV_SD(float, 4, 2, 11); else CKV_SD(float, 4, 6, 5); }
         else if (G == 2) { if (U == 4) CKV_SD(float, 2, 4, 6); else CKV_SD(float, 2, 9, 7); }
         else { if (U == 4) CKV_SD(float, 1, 4, 8); else CKV_SD(float, 1, 9, 9); }
     }

@@ -9,16 +9,20 @@
 //              fixed fp32 order of k_score and writes the 64-bit rank key
 //              (descending score, ascending id) into every CTA's key table
 //   -- cluster barrier
-//   2. rank    CTA r ranks clusters c = r (mod NC), one warp per cluster,
-//              the 32 lanes counting smaller keys, and writes
-//              (order[rank] = c, size[rank] = n_c) into every CTA
-//   -- cluster barrier
-//   3. fill    every CTA prefix-sums the sizes in rank order (redundantly, no
-//              leader round trip); sel_cnt = min(budget, total)
+//   2. select  every CTA finds, on its own copy of the keys, the cluster at
+//              which the running size sum in rank order reaches the budget:
+//              a weighted radix select (8-bit digits from the top of the key,
+//              per-digit size sums and counts by 32-bit shared atomics, the
+//              first digit whose running size sum reaches the budget kept)
+//   3. fill    the non-empty clusters up to that key are compacted; each
+//              one's rank and first row among them come from counting the
+//              smaller keys and summing their sizes; sel_cnt =
+//              min(budget, total). No cluster barrier: all CTAs agree
 //   4. resolve CTA r owns rows [r*chunk, (r+1)*chunk) of the attended list
 //              (sinks, recalled, recent); each recalled row finds its rank by
-//              binary search and its position through offsets/perm; the
-//              positions go to shared memory and to sel_idx (ABI output)
+//              binary search over the selected clusters and its position
+//              through offsets/perm (perm loads batched); the positions go to
+//              shared memory and to sel_idx (ABI output)
 //   5. attend  split-K online softmax over the CTA's rows (half-warp per
 //              256-byte row, U rows in flight per half-warp, U chosen so a
 //              CTA's rows arrive in one batch at the usual shapes), merged
@@ -72,7 +76,7 @@ struct Args {
 
 // dynamic shared memory layout (bytes), sized by C_cap, G and chunk
 struct Layout {
-    size_t keys, order, size, start, offs, pos, mo, ml, part, total;
+    size_t keys, lkey, csz, lst, order, size, start, offs, pos, mo, ml, part, total;
 };
 
 __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -81,8 +85,11 @@ __host__ __device__ inline Layout layout(int C_cap, int G, int chunk, int nc) {
     Layout L;
     size_t o = 0;
     L.keys = o;   o += al16((size_t)C_cap * 8);
+    L.lkey = o;   o += al16((size_t)C_cap * 8);           // keys of the selected clusters
+    L.csz = o;    o += al16((size_t)C_cap * 4);           // cluster sizes by id
+    L.lst = o;    o += al16((size_t)C_cap * 4);           // selected cluster ids (unordered)
     L.order = o;  o += al16((size_t)C_cap * 4);
-    L.size = o;   o += al16((size_t)C_cap * 4);
+    L.size = o;   o += al16((size_t)C_cap * 4);           // sizes of the selected clusters
     L.start = o;  o += al16((size_t)(C_cap + 1) * 4);
     L.offs = o;   o += al16((size_t)(C_cap + 1) * 4);     // the problem's offsets row
     L.pos = o;    o += al16((size_t)chunk * 4);
@@ -104,15 +111,20 @@ k_select_decode(const Args a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const Layout LY = layout(a.C_cap, G, a.chunk, nc);
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem + LY.keys);
+    uint64_t *lkey = reinterpret_cast<uint64_t *>(smem + LY.lkey);
+    int32_t *csz = reinterpret_cast<int32_t *>(smem + LY.csz);
+    int32_t *lst = reinterpret_cast<int32_t *>(smem + LY.lst);
     int32_t *order = reinterpret_cast<int32_t *>(smem + LY.order);
-    int32_t *rsz = reinterpret_cast<int32_t *>(smem + LY.size);
+    int32_t *lsz = reinterpret_cast<int32_t *>(smem + LY.size);
     int32_t *start = reinterpret_cast<int32_t *>(smem + LY.start);
     int32_t *off_s = reinterpret_cast<int32_t *>(smem + LY.offs);
     int32_t *pos_s = reinterpret_cast<int32_t *>(smem + LY.pos);
     float *mo = reinterpret_cast<float *>(smem + LY.mo);
     float *mml = reinterpret_cast<float *>(smem + LY.ml);
     float *part = reinterpret_cast<float *>(smem + LY.part);
-    __shared__ int wsum[WARPS];
+    __shared__ __align__(16) unsigned s_hw[2][256];  // size sum per digit
+    __shared__ __align__(16) unsigned s_hn[2][256];  // cluster count per digit
+    __shared__ int s_before, s_total, s_bin, s_cnt, s_m;
 
     const int nC = min(max(a.ncl[p], 0), a.C_cap);
     const int32_t *off = a.offsets + (size_t)p * (a.C_cap + 1);
@@ -121,6 +133,9 @@ k_select_decode(const Args a) {
 
     // the problem's offsets row, needed by ranking and by position lookup
     for (int i = tid; i <= nC; i += THREADS) off_s[i] = off[i];
+    s_hw[0][tid] = 0;  // THREADS == 256
+    s_hn[0][tid] = 0;
+    if (tid == 0) s_m = 0;
     cl.sync();  // every CTA of the cluster is running before any DSMEM access
 
     // ---- 1. score (fixed fp32 order), keys broadcast to every CTA ----
@@ -161,60 +176,132 @@ k_select_decode(const Args a) {
     }
     cl.sync();
 
-    // ---- 2. rank own clusters (c = rank mod nc): one warp per cluster ----
-    for (int c = rank + warp * nc; c < nC; c += WARPS * nc) {  // warp-uniform
-        const uint64_t kc = keys[c];
-        int n0 = 0, n1 = 0, n2 = 0, n3 = 0;  // independent partial counts
-        int k = lane;
-        for (; k + 96 < nC; k += 128) {
-            n0 += keys[k] < kc;
-            n1 += keys[k + 32] < kc;
-            n2 += keys[k + 64] < kc;
-            n3 += keys[k + 96] < kc;
-        }
-        for (; k < nC; k += 32) n0 += keys[k] < kc;
-        const int r = __reduce_add_sync(FULL, n0 + n1 + n2 + n3);
-        int sz = 0;
-        const int o0 = off_s[c], o1 = off_s[c + 1];
-        if (o0 < 0 || o1 < o0 || o1 > a.perm_cap) {
-            if (lane == 0) dev_flag(CKV_DEVERR_OFFSETS);
-        } else {
-            sz = o1 - o0;
-        }
-        if (lane < nc) {  // every CTA gets (order, size)
-            *cl.map_shared_rank(&order[r], lane) = c;
-            *cl.map_shared_rank(&rsz[r], lane) = sz;
-        }
-    }
-    cl.sync();
-
-    // ---- 3. fill: exclusive scan of sizes in rank order (every CTA) ----
-    {
-        const int per = (nC + THREADS - 1) / THREADS;
-        const int b = tid * per, e = min(nC, b + per);
-        int loc = 0;
-        for (int r = b; r < e; ++r) loc += rsz[r];
-        int incl = loc;
+    // ---- 2. threshold: the cluster at which the running size sum, in rank
+    // order, reaches the budget. Weighted radix select over the 64-bit keys,
+    // 8-bit digits from the top; the id half holds c < 2^16, so its two upper
+    // bytes are zero for every key and are skipped. Every CTA runs it on its
+    // own copy of the key table. ----
+    uint64_t pre = 0, msk = 0;  // key bits fixed so far
+    int need = a.B;             // budget still to reach inside the fixed prefix
+    bool take_all = false;      // the sizes sum to less than the budget
+    if (a.B > 0) {
+        constexpr int NPASS = 6;
+        for (int ps = 0; ps < NPASS; ++ps) {
+            const int sh = ps < 4 ? 56 - 8 * ps : 8 * (NPASS - 1 - ps);
+            unsigned *hw = s_hw[ps & 1], *hn = s_hn[ps & 1];
+            // plain 32-bit shared atomics: (weight, count) per digit
+            for (int c = tid; c < nC; c += THREADS) {
+                const uint64_t k = keys[c];
+                int sz;
+                if (ps == 0) {
+                    const int o0 = off_s[c], o1 = off_s[c + 1];
+                    sz = 0;
+                    if (o0 < 0 || o1 < o0 || o1 > a.perm_cap) dev_flag(CKV_DEVERR_OFFSETS);
+                    else sz = o1 - o0;
+                    csz[c] = sz;
+                } else {
+                    sz = csz[c];
+                }
+                if ((k & msk) == pre) {
+                    const int dg = (int)((k >> sh) & 255);
+                    atomicAdd(&hw[dg], (unsigned)sz);
+                    atomicAdd(&hn[dg], 1u);
+                }
+            }
+            s_hw[(ps + 1) & 1][tid] = 0;  // the next pass's tables (THREADS == 256)
+            s_hn[(ps + 1) & 1][tid] = 0;
+            __syncthreads();
+            if (warp == 0) {
+                // lane l owns digits 8l..8l+7: the first digit whose running
+                // weight reaches `need`. Valid offsets keep every sum below
+                // perm_cap < 2^31.
+                const uint4 wa = reinterpret_cast<const uint4 *>(hw)[lane * 2];
+                const uint4 wb = reinterpret_cast<const uint4 *>(hw)[lane * 2 + 1];
+                const unsigned wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                unsigned wl = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(FULL, incl, o);
-            if (lane >= o) incl += t;
+                for (int i = 0; i < 8; ++i) wl += wv[i];
+                unsigned incl = wl;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned t = __shfl_up_sync(FULL, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                if (ps == 0 && lane == 31) s_total = (int)incl;
+                const unsigned hit = __ballot_sync(FULL, incl >= (unsigned)need);
+                if (hit == 0) {
+                    if (lane == 0) s_bin = -1;
+                } else if (lane == __ffs(hit) - 1) {
+                    unsigned before = incl - wl;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (before + wv[i] >= (unsigned)need) {
+                            s_bin = lane * 8 + i;
+                            s_before = (int)before;
+                            s_cnt = (int)hn[lane * 8 + i];
+                            break;
+                        }
+                        before += wv[i];
+                    }
+                }
+            }
+            __syncthreads();
+            const int bin = s_bin;
+            if (bin < 0) {
+                take_all = true;
+                break;
+            }
+            pre |= (uint64_t)bin << sh;
+            msk |= 255ull << sh;
+            need -= s_before;
+            if (s_cnt == 1) break;
         }
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
-        int wpre = 0;
-        for (int w = 0; w < warp; ++w) wpre += wsum[w];
-        int run = wpre + incl - loc;
-        for (int r = b; r < e; ++r) {
-            start[r] = run;
-            run += rsz[r];
-        }
-        if (tid == THREADS - 1) start[nC] = run;  // total
-        __syncthreads();
     }
-    const int total = start[nC];
+    const int total = a.B > 0 ? s_total : 0;
     const int cnt = min(a.B, total);
     if (rank == 0 && tid == 0) a.sel_cnt[p] = cnt;
+
+    // ---- 3. the selected non-empty clusters (every key up to the threshold),
+    // compacted, then each one's rank and start row among them by counting
+    // the smaller keys (thread per selected cluster, broadcast reads) ----
+    if (a.B > 0) {
+        for (int c0 = warp * 32; c0 < nC; c0 += THREADS) {  // warp-uniform
+            const int c = c0 + lane;
+            uint64_t k = 0;
+            int sz = 0;
+            bool in = false;
+            if (c < nC) {
+                k = keys[c];
+                sz = csz[c];
+                in = sz > 0 && (take_all || (k & msk) <= pre);
+            }
+            const unsigned bal = __ballot_sync(FULL, in);
+            int base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&s_m, __popc(bal));
+            base = __shfl_sync(FULL, base, 0);
+            if (in) {
+                const int i = base + __popc(bal & lanemask_lt());
+                lst[i] = c;
+                lkey[i] = k;
+                lsz[i] = sz;
+            }
+        }
+    }
+    __syncthreads();
+    const int nsel = s_m;
+    for (int i = tid; i < nsel; i += THREADS) {
+        const uint64_t ki = lkey[i];
+        int r = 0, st = 0;
+        for (int j = 0; j < nsel; ++j) {
+            if (lkey[j] < ki) {
+                ++r;
+                st += lsz[j];
+            }
+        }
+        order[r] = lst[i];
+        start[r] = st;
+    }
+    __syncthreads();
 
     // ---- 4. resolve this CTA's rows of the attended list ----
     const int tb = a.tail_b[p];
@@ -222,31 +309,45 @@ k_select_decode(const Args a) {
     const int n_att = a.S + cnt + ntail;
     if (rank == 0 && tid == 0 && n_att > nc * a.chunk) dev_flag(CKV_DEVERR_INDEX);
     const int j0 = rank * a.chunk, j1 = min(n_att, j0 + a.chunk);
-    for (int j = j0 + tid; j < j1; j += THREADS) {
-        int row;
-        if (j < a.S) {
-            row = j;
-        } else if (j < a.S + cnt) {
-            const int k = j - a.S;
-            // last rank r with start[r] <= k (a non-empty cluster)
-            int lo = 0, hi = nC - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (start[mid] <= k) lo = mid;
-                else hi = mid - 1;
+    constexpr int RB = 4;  // rows per thread whose perm loads are in flight together
+    for (int jb = j0 + tid; jb < j1; jb += THREADS * RB) {
+        int slot[RB];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int j = jb + u * THREADS;
+            slot[u] = -1;
+            if (j < j1 && j >= a.S && j < a.S + cnt) {
+                const int k = j - a.S;
+                // last rank r with start[r] <= k (every listed cluster is non-empty)
+                int lo = 0, hi = nsel - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (start[mid] <= k) lo = mid;
+                    else hi = mid - 1;
+                }
+                slot[u] = off_s[order[lo]] + (k - start[lo]);
             }
-            const int c = order[lo];
-            const int slot = off_s[c] + (k - start[lo]);
-            row = (slot >= 0 && slot < a.perm_cap) ? pp[slot] : -1;
-            a.sel_idx[(size_t)p * a.B + k] = row;
-        } else {
-            row = tb + (j - a.S - cnt);
         }
-        if (row < 0 || row >= a.kv_rows) {
-            dev_flag(CKV_DEVERR_INDEX);
-            row = -1;
+        int row[RB];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int j = jb + u * THREADS;
+            if (j < a.S) row[u] = j;
+            else if (j < a.S + cnt) row[u] = (slot[u] >= 0 && slot[u] < a.perm_cap) ? __ldg(pp + slot[u]) : -1;
+            else row[u] = tb + (j - a.S - cnt);
         }
-        pos_s[j - j0] = row;
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int j = jb + u * THREADS;
+            if (j >= j1) break;
+            int r = row[u];
+            if (j >= a.S && j < a.S + cnt) a.sel_idx[(size_t)p * a.B + (j - a.S)] = r;
+            if (r < 0 || r >= a.kv_rows) {
+                dev_flag(CKV_DEVERR_INDEX);
+                r = -1;
+            }
+            pos_s[j - j0] = r;
+        }
     }
     __syncthreads();
 

@@ -17,16 +17,21 @@ pytestmark = pytest.mark.gpu
 
 
 def _case(dev, dtype, P, G, C, n, budget, L, S, tails, seed, ties=False, n_clusters=None,
-          skew=0.8, q_scale=1.0):
+          skew=0.8, q_scale=1.0, all_equal=False, singletons=False):
     rng = np.random.default_rng(seed)
     mode = mode_of(dtype)
     d = 128
     tb0 = S
     C_cap, perm_cap = C + 3, n + 5
     lab = synth.random_labels(P, n, C, seed=seed, skew=skew).numpy()
+    if singletons:  # every token its own cluster
+        assert C == n
+        lab = np.stack([rng.permutation(n) for _ in range(P)]).astype(np.int32)
     mu = rng.standard_normal((P, C, d)) * 0.3
     if ties:
         mu[:, 1::3] = mu[:, 0:-1:3][:, :mu[:, 1::3].shape[1]]
+    if all_equal:  # one score for every cluster: the id order decides alone
+        mu[:] = mu[:, :1]
     mu_lp = oracle.round_to(mu, mode).astype(np.float32)
     q = oracle.round_to(rng.standard_normal((P, G, d)) * q_scale, mode).astype(np.float32)
     K = oracle.round_to(rng.standard_normal((P, L, d)) * 0.5, mode).astype(np.float32)
@@ -95,12 +100,15 @@ def test_fused_step_ties_large_C_partial_counts_no_sinks(cuda_device):
     assert ckv.ckv_device_error() == 0
 
 
-def test_fused_step_many_problems_single_cta_clusters(cuda_device):
-    # enough problems that each cluster is a single CTA
+@pytest.mark.parametrize("G,dtype", [(1, torch.bfloat16), (2, torch.bfloat16),
+                                     (4, torch.bfloat16), (4, torch.float32)])
+def test_fused_step_many_problems_single_cta_clusters(cuda_device, G, dtype):
+    # enough problems that each cluster is a single CTA (the many-problem
+    # instantiations with fewer rows in flight)
     P, L, S = 700, 1500, 4
     tails = [(1400, 1400 + (p % 64)) for p in range(P)]
-    refs, sel, cnt, out, _ = _case(cuda_device, torch.bfloat16, P, 1, C=40, n=1300, budget=256,
-                                   L=L, S=S, tails=tails, seed=11)
+    refs, sel, cnt, out, _ = _case(cuda_device, dtype, P, G, C=40, n=1300, budget=256,
+                                   L=L, S=S, tails=tails, seed=11 + G)
     _check(refs, sel, cnt, out)
     assert ckv.ckv_device_error() == 0
 
@@ -124,3 +132,31 @@ def test_fused_step_equals_separate_calls(cuda_device):
     assert np.array_equal(cnt2.cpu().numpy(), cnt)
     assert np.array_equal(sel2.cpu().numpy(), sel)
     assert np.abs(out2.cpu().numpy() - out).max() <= 1e-5
+
+
+@pytest.mark.parametrize("budget", [1, 777, 3900])
+def test_fused_step_all_scores_equal(cuda_device, budget):
+    # identical centroids: the selection is decided by cluster id alone
+    # (budget 3900 equals the clustered total exactly)
+    P, L, S = 3, 5000, 16
+    tails = [(4936, 5000)] * P
+    refs, sel, cnt, out, _ = _case(cuda_device, torch.bfloat16, P, 2, C=400, n=3900,
+                                   budget=budget, L=L, S=S, tails=tails, seed=21,
+                                   all_equal=True)
+    _check(refs, sel, cnt, out)
+    assert ckv.ckv_device_error() == 0
+
+
+@pytest.mark.parametrize("P,C", [(2, 4000), (600, 1100)])
+def test_fused_step_singleton_clusters(cuda_device, P, C):
+    # C = n: every cluster holds one token, so the budget selects 1024
+    # clusters, the top-B tokens by q . k (the largest selected set); 600
+    # problems make every problem a single CTA
+    S = 4
+    L = S + C + 64
+    tails = [(S + C, S + C + (p % 50)) for p in range(P)]
+    refs, sel, cnt, out, _ = _case(cuda_device, torch.bfloat16, P, 1, C=C, n=C,
+                                   budget=1024, L=L, S=S, tails=tails, seed=23,
+                                   singletons=True)
+    _check(refs, sel, cnt, out)
+    assert ckv.ckv_device_error() == 0
