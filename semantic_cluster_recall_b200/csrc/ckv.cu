@@ -199,6 +199,76 @@ void decode_shape(int P, int max_rows, int sms, int *chunk, int *nsplit) {
     *nsplit = (max_rows + c - 1) / c;
 }
 
+// instantiations of the fused step: (kernel, smem_optin slot)
+struct sd_kernel {
+    const void *fn;
+    int slot;
+};
+
+template <typename T, int G, int U>
+sd_kernel sd_entry(int slot) {
+    return {reinterpret_cast<const void *>(&sd::k_select_decode<T, G, U>), SLOT_SD_BASE + slot};
+}
+
+sd_kernel sd_pick(ckv_dtype dt, int G, int U) {
+    if (dt == CKV_BF16) {
+        if (G == 4) return U == 2 ? sd_entry<bf16, 4, 2>(10) : sd_entry<bf16, 4, 6>(0);
+        if (G == 2) return U == 4 ? sd_entry<bf16, 2, 4>(1) : sd_entry<bf16, 2, 9>(2);
+        return U == 4 ? sd_entry<bf16, 1, 4>(3) : sd_entry<bf16, 1, 9>(4);
+    }
+    if (G == 4) return U == 2 ? sd_entry<float, 4, 2>(11) : sd_entry<float, 4, 6>(5);
+    if (G == 2) return U == 4 ? sd_entry<float, 2, 4>(6) : sd_entry<float, 2, 9>(7);
+    return U == 4 ? sd_entry<float, 1, 4>(8) : sd_entry<float, 1, 9>(9);
+}
+
+cudaError_t sd_optin(const sd_kernel &k, size_t smem) {
+    return smem_optin(k.fn, smem, k.slot);
+}
+
+// How many thread-block clusters of nc CTAs (smem bytes each) the device
+// holds at once; cached per (device, instantiation, nc, smem).
+cudaError_t sd_clusters_per_wave(const sd_kernel &k, int nc, size_t smem, int *out) {
+    struct Entry {
+        int dev, slot, nc;
+        size_t smem;
+        int fit;
+    };
+    static std::mutex mu;
+    static Entry cache[256];
+    static int n_cache = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (int i = 0; i < n_cache; ++i)
+            if (cache[i].dev == dev && cache[i].slot == k.slot && cache[i].nc == nc &&
+                cache[i].smem == smem) {
+                *out = cache[i].fit;
+                return cudaSuccess;
+            }
+    }
+    cudaError_t e = sd_optin(k, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nc, 1, 1);
+    cfg.blockDim = dim3(sd::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int fit = 0;
+    e = cudaOccupancyMaxActiveClusters(&fit, k.fn, &cfg);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(mu);
+    if (n_cache < 256) cache[n_cache++] = {dev, k.slot, nc, smem, fit};
+    *out = fit;
+    return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -440,19 +510,48 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
     const int64_t max_rows64 = (int64_t)sink + budget + max_tail;
     if (max_rows64 > (1 << 30)) return fail(CKV_ERR_INVALID, "too many attended rows");
     const int max_rows = max_rows64 < 1 ? 1 : (int)max_rows64;
-    const int sms = sm_count();
-    int nc = (4 * sms + P - 1) / P;
-    nc = nc < 1 ? 1 : (nc > sd::NC_MAX ? sd::NC_MAX : nc);
-    int chunk = (max_rows + nc - 1) / nc;
-    if (chunk > sd::POS_MAX)
-        return fail(CKV_ERR_UNSUPPORTED, "fused step supports up to %d attended rows per problem",
-                    sd::NC_MAX * sd::POS_MAX);
-    const size_t smem = sd::layout(C_cap, G, chunk, nc).total;
-    // rows in flight per half-warp: one batch for the CTA's rows when the
-    // registers allow it (16 half-warps per CTA); when a problem is a single
-    // CTA (many problems), fewer rows and registers, so that 4 CTAs share an
-    // SM and their selection phases overlap each other's gathers
-    const int U = (G == 4) ? (nc == 1 ? 2 : 6) : ((chunk <= 16 * 4 || nc == 1) ? 4 : 9);
+    // CTAs per problem (nc) and rows in flight per half-warp (U): the largest
+    // cluster size whose launch fits the GPU in one wave (all P clusters
+    // resident at once), with U chosen so that a CTA's rows arrive in one
+    // batch at the usual shapes. When not even one CTA per problem fits in a
+    // wave (many problems), one CTA per problem with fewer rows in flight and
+    // registers, so that more CTAs share an SM and their selection phases
+    // overlap each other's gathers.
+    int nc = 0, U = 0, chunk = 0;
+    size_t smem = 0;
+    sd_kernel kern = {nullptr, 0};
+    cudaError_t e = cudaSuccess;
+    for (int cand = sd::NC_MAX; cand >= 1; cand >>= 1) {
+        const int ch = (max_rows + cand - 1) / cand;
+        if (ch > sd::POS_MAX) break;
+        const int u = (G == 4) ? 6 : (ch <= 16 * 4 ? 4 : 9);
+        const sd_kernel k = sd_pick(dt, G, u);
+        const size_t sm = sd::layout(C_cap, G, ch, cand).total;
+        int fit = 0;
+        if (sd_clusters_per_wave(k, cand, sm, &fit) != cudaSuccess) {
+            cudaGetLastError();  // not a launchable shape: try fewer CTAs per problem
+            fit = 0;
+        }
+        if (fit >= P || cand == 1) {
+            nc = cand; chunk = ch; smem = sm; U = u; kern = k;
+            if (fit < P && cand == 1) {  // more than one wave even at one CTA per problem
+                U = (G == 4) ? 2 : 4;
+                kern = sd_pick(dt, G, U);
+            }
+            break;
+        }
+    }
+    if (nc == 0) {  // the rows do not fit one CTA: the smallest nc that holds them
+        nc = (max_rows + sd::POS_MAX - 1) / sd::POS_MAX;
+        nc = nc <= 2 ? nc : (nc <= 4 ? 4 : 8);
+        chunk = (max_rows + nc - 1) / nc;
+        if (chunk > sd::POS_MAX)
+            return fail(CKV_ERR_UNSUPPORTED, "fused step supports up to %d attended rows per problem",
+                        sd::NC_MAX * sd::POS_MAX);
+        U = (G == 4) ? 6 : 9;
+        kern = sd_pick(dt, G, U);
+        smem = sd::layout(C_cap, G, chunk, nc).total;
+    }
     sd::Args a;
     a.q = q;
     a.lp = centroids_lp;
@@ -486,22 +585,11 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaSuccess;
-#define CKV_SD(T, GG, UU, SLOT)                                                            \
-    do {                                                                                   \
-        e = smem_optin(sd::k_select_decode<T, GG, UU>, smem, SLOT_SD_BASE + (SLOT));       \
-        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sd::k_select_decode<T, GG, UU>, a); \
-    } while (0)
-    if (dt == CKV_BF16) {
-        if (G == 4) { if (U == 2) CKV_SD(bf16, 4, 2, 10); else CKV_SD(bf16, 4, 6, 0); }
-        else if (G == 2) { if (U == 4) CKV_SD(bf16, 2, 4, 1); else CKV_SD(bf16, 2, 9, 2); }
-        else { if (U == 4) CKV_SD(bf16, 1, 4, 3); else CKV_SD(bf16, 1, 9, 4); }
-    } else {
-        if (G == 4) { if (U == 2) CKV_SD(float, 4, 2, 11); else CKV_SD(float, 4, 6, 5); }
-        else if (G == 2) { if (U == 4) CKV_SD(float, 2, 4, 6); else CKV_SD(float, 2, 9, 7); }
-        else { if (U == 4) CKV_SD(float, 1, 4, 8); else CKV_SD(float, 1, 9, 9); }
+    e = sd_optin(kern, smem);
+    if (e == cudaSuccess) {
+        void *args[] = {&a};
+        e = cudaLaunchKernelExC(&cfg, kern.fn, args);
     }
-#undef CKV_SD
     if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "k_select_decode: %s", cudaGetErrorString(e));
     return launched("k_select_decode");
 }

@@ -131,14 +131,15 @@ k_select_decode(const Args a) {
     const int32_t *pp = a.perm + (size_t)p * a.perm_cap;
     const T *qp = reinterpret_cast<const T *>(a.q) + (size_t)p * G * D;
 
-    // the problem's offsets row, needed by ranking and by position lookup
+    // the problem's offsets row, needed by selection and by position lookup
     for (int i = tid; i <= nC; i += THREADS) off_s[i] = off[i];
     s_hw[0][tid] = 0;  // THREADS == 256
     s_hn[0][tid] = 0;
     if (tid == 0) s_m = 0;
-    cl.sync();  // every CTA of the cluster is running before any DSMEM access
 
-    // ---- 1. score (fixed fp32 order), keys broadcast to every CTA ----
+    // ---- 1. score (fixed fp32 order), keys broadcast to every CTA. The
+    // first batch of centroid rows is loaded and scored before the cluster
+    // barrier (only the DSMEM writes must wait for it) ----
     {
         float4 qv[G];
 #pragma unroll
@@ -146,7 +147,8 @@ k_select_decode(const Args a) {
         const T *lpp = reinterpret_cast<const T *>(a.lp) + (size_t)p * a.C_cap * D + lane * 4;
         const int cstride = nc * WARPS;
         constexpr int SB = 8;  // centroid rows in flight per warp
-        for (int cb = rank * WARPS + warp; cb < nC; cb += cstride * SB) {
+        uint64_t kk[SB];
+        auto score_batch = [&](int cb) {
             float4 mrow[SB];
 #pragma unroll
             for (int u = 0; u < SB; ++u) {
@@ -155,8 +157,6 @@ k_select_decode(const Args a) {
             }
 #pragma unroll
             for (int u = 0; u < SB; ++u) {
-                const int c = cb + u * cstride;
-                if (c >= nC) break;  // warp-uniform
                 float tot = 0.f;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
@@ -169,9 +169,21 @@ k_select_decode(const Args a) {
                     for (int o = 16; o >= 1; o >>= 1) sc = sc + __shfl_xor_sync(FULL, sc, o);
                     tot = (g == 0) ? sc : tot + sc;
                 }
-                const uint64_t key = ((uint64_t)(~ordered_bits(tot)) << 32) | (uint32_t)c;
-                if (lane < nc) *cl.map_shared_rank(&keys[c], lane) = key;
+                kk[u] = ((uint64_t)(~ordered_bits(tot)) << 32) | (uint32_t)(cb + u * cstride);
             }
+        };
+        int cb = rank * WARPS + warp;
+        score_batch(cb);
+        cl.sync();  // every CTA of the cluster is running before any DSMEM access
+        for (;;) {  // warp-uniform
+#pragma unroll
+            for (int u = 0; u < SB; ++u) {
+                const int c = cb + u * cstride;
+                if (c < nC && lane < nc) *cl.map_shared_rank(&keys[c], lane) = kk[u];
+            }
+            cb += cstride * SB;
+            if (cb >= nC) break;
+            score_batch(cb);
         }
     }
     cl.sync();

@@ -82,7 +82,8 @@ class Workload:
 
 SEED_BASE = 0xC1A5
 
-# The five workloads. Problem index p = ((layer * batch + b) * heads_kv + h).
+# The five workloads, and one profiling stand-in. Problem index
+# p = ((layer * batch + b) * heads_kv + h).
 WORKLOADS = {
     # Tiny single head, fp32, 32-component mixture.
     "tiny_f32": Workload("tiny_f32", P=1, G=1, L=2048, d=128, dtype="f32", S=4, W=32,
@@ -105,6 +106,13 @@ WORKLOADS = {
     "long_128k": Workload("long_128k", P=32, G=4, L=131072, d=128, dtype="bf16",
                           S=16, W=128, C=1600, T=8, B=2048, M=1600, steps=64,
                           batch=4, heads_kv=8, seed=SEED_BASE + 5),
+    # Profiling stand-in for the many-problem decode (a problem per CTA):
+    # 8 layers x batch 4 x 32 KV heads at 8k context, clusters of the same
+    # average size (C = 100), so a capture holds ~4.5 GB instead of 69 GB.
+    "llama2_8layer_8k_decode": Workload("llama2_8layer_8k_decode", P=8 * 4 * 32, G=1, L=8192,
+                                        d=128, dtype="bf16", S=16, W=64, C=100, T=10, B=1024,
+                                        M=100, layers=8, batch=4, heads_kv=32,
+                                        seed=SEED_BASE + 6),
 }
 
 WORKLOAD_ORDER = ["tiny_f32", "llama2_layer_32k", "llama3_gqa_32k",
