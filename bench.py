@@ -286,6 +286,9 @@ def decode_32layer(dev, stream, n_steps: int = 20) -> dict:
         times.append(e0.elapsed_time(e1) * 1e-3)
     del g
     loop = {f"per_layer_P{pl}": layer_loop(w, st, q, K, V, pl, stream, pk) for pl in (32, 128)}
+    del st
+    torch.cuda.empty_cache()
+    overlap = incremental_overlap(w, K, V, q, dev)
     t = statistics.median(times)
     byts = decode_bytes(w.replace(tail_cap=0))
     res = {"workload": w.name, "P": w.P, "steps_per_s": 1.0 / t, "us_per_step": t * 1e6,
@@ -296,10 +299,24 @@ def decode_32layer(dev, stream, n_steps: int = 20) -> dict:
            "prefill_clustering": {"keys_per_s": w.P * w.N / t_cluster,
                                   "ms": t_cluster * 1e3, "keys": w.P * w.N},
            "launch": "fused select + sparse decode, CUDA graph replay, L2 flushed",
-           "layer_loop": loop}
-    del K, V, st, flush
+           "layer_loop": loop, "incremental_overlap": overlap}
+    del K, V, flush
     torch.cuda.empty_cache()
     return res
+
+
+def layer_launches(w: synth.Workload, st: ClusterRecall, q, K, V, per_layer: int, stream):
+    """One decode step of every layer: a fused launch over the first
+    `per_layer` problems of each layer's w.P // w.layers."""
+    per_l = w.P // w.layers
+    for l in range(w.layers):
+        a, b = l * per_l, l * per_l + per_layer
+        ckv.ckv_select_decode(q[a:b], st.centroids_lp[a:b], st.n_clusters[a:b], st.C_cap,
+                              st.offsets[a:b], st.perm[a:b], st.perm_cap, st.B,
+                              st.sel_idx[a:b], st.sel_cnt[a:b], K[a:b], V[a:b], K.stride(0),
+                              st.kv_rows, st.S, st.tail_begin[a:b], st.tail_end[a:b],
+                              st.max_tail, st.scale, st.out[a:b], P=per_layer, G=st.G,
+                              d=st.d, stream=stream)
 
 
 def layer_loop(w: synth.Workload, st: ClusterRecall, q, K, V, per_layer: int, stream, pk,
@@ -310,18 +327,10 @@ def layer_loop(w: synth.Workload, st: ClusterRecall, q, K, V, per_layer: int, st
     launches read different layers' data (32 x the per-layer bytes, far above
     the L2 size), so no flush is needed; the time per step is the replay time
     / 32, without a per-step launch gap."""
-    per_l = w.P // w.layers
     gr = torch.cuda.CUDAGraph()
 
     def launches():
-        for l in range(w.layers):
-            a, b = l * per_l, l * per_l + per_layer
-            ckv.ckv_select_decode(q[a:b], st.centroids_lp[a:b], st.n_clusters[a:b], st.C_cap,
-                                  st.offsets[a:b], st.perm[a:b], st.perm_cap, st.B,
-                                  st.sel_idx[a:b], st.sel_cnt[a:b], K[a:b], V[a:b], K.stride(0),
-                                  st.kv_rows, st.S, st.tail_begin[a:b], st.tail_end[a:b],
-                                  st.max_tail, st.scale, st.out[a:b], P=per_layer, G=st.G,
-                                  d=st.d, stream=stream)
+        layer_launches(w, st, q, K, V, per_layer, stream)
 
     launches()  # warm-up outside the capture
     torch.cuda.synchronize()
@@ -344,6 +353,73 @@ def layer_loop(w: synth.Workload, st: ClusterRecall, q, K, V, per_layer: int, st
             "roofline": {"bound": "hbm", "achieved": byts / t / 1e9, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": byts / t / 1e9 / pk["hbm_gbs"],
                          "peak_source": pk["source"] + " copy"}}
+
+
+def incremental_overlap(w: synth.Workload, K, V, q, dev, n_steps: int = 8,
+                        caps=(0, 16, 64)) -> dict:
+    """Clustering of generated tokens hidden behind decode. The last tail_cap
+    prompt tokens stand for a full tail; its oldest tail_cap - W tokens of all
+    4096 problems are clustered into inc_C more clusters (inc_T rounds),
+    either synchronously after n_steps model decode steps (each step = one
+    fused launch per layer over that layer's 128 problems, as a model runs
+    them) or in the background: started on a low-priority side stream before
+    the steps, the tensor-core assignment held to max_sms SMs, and published
+    after them. Each mode ends with one more step that sees the published
+    clusters. CUDA events on the high-priority main stream; best of 3 runs."""
+    main = torch.cuda.Stream(device=dev, priority=-1)
+    side = torch.cuda.Stream(device=dev, priority=0)
+    n_inc = w.tail_cap - w.W
+    n_pre = w.L - w.S - w.tail_cap
+    per_layer = w.P // w.layers
+    st = ClusterRecall(w.P, w.G, w.d, w.torch_dtype, w.L, w.S, w.B, w.C + w.inc_C,
+                       n_pre + n_inc, w.tail_cap, dev, stream=main)
+    with torch.cuda.stream(main):
+        st.prefill(K, w.L, w.tail_cap, w.C, w.T)
+
+    def reset():
+        st.C_used, st.n_clustered, st.tail_lo = w.C, n_pre, w.L - w.tail_cap
+        with torch.cuda.stream(main):
+            st.n_clusters.fill_(w.C)
+            st.tail_begin.fill_(w.L - w.tail_cap)
+        torch.cuda.synchronize()
+
+    def run(mode: str, cap: int = 0) -> float:
+        best = float("inf")
+        for _ in range(3):
+            reset()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(main):
+                e0.record(main)
+                if mode == "background":
+                    st.incremental_begin(K, n_inc, w.inc_C, w.inc_T, side, max_sms=cap)
+                if mode != "cluster":
+                    for _ in range(n_steps):
+                        layer_launches(w, st, q, K, V, per_layer, main)
+                if mode in ("sync", "cluster"):
+                    st.incremental(K, n_inc, w.inc_C, w.inc_T)
+                if mode == "background":
+                    st.incremental_commit()
+                if mode != "cluster":
+                    layer_launches(w, st, q, K, V, per_layer, main)
+                e1.record(main)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return best
+
+    t_dec, t_cl, t_sync = run("decode"), run("cluster"), run("sync")
+    bg = {str(c): run("background", c) for c in caps}
+    assert int(st.n_clusters[0]) == w.C + w.inc_C
+    cap_best = min(bg, key=bg.get)
+    res = {"decode_steps": n_steps + 1, "launches_per_step": w.layers,
+           "problems_per_launch": per_layer, "clustered_tokens_per_problem": n_inc,
+           "new_clusters": w.inc_C, "rounds": w.inc_T,
+           "decode_alone_ms": t_dec, "clustering_alone_ms": t_cl, "sync_ms": t_sync,
+           "background_ms_by_max_sms": bg, "best_max_sms": int(cap_best),
+           "hidden_fraction": (t_sync - bg[cap_best]) / t_cl}
+    del st
+    torch.cuda.empty_cache()
+    return res
 
 
 def e2e_measure(w: synth.Workload, dev, stream, steps: int):

@@ -133,6 +133,29 @@ ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_st
                        int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
                        size_t ws_bytes, void *stream);
 
+/* ckv_cluster for background use beside other GPU work ("IV.B Semantic
+ * Clustering": clustering is launched asynchronously and overlaps other
+ * inference kernels). Identical arguments and results, plus
+ *   max_sms   upper bound on the SMs the persistent tensor-core assignment
+ *             kernel occupies (0 = all); the other clustering kernels are
+ *             short-lived CTAs that interleave with other streams' work, so
+ *             running this on a low-priority stream leaves the remaining SMs
+ *             to the caller's high-priority kernels.
+ * Clustering into cluster slots [cluster_base, cluster_base + C) and perm
+ * slots [perm_base, perm_base + n_tok) beyond a problem's n_clusters does not
+ * disturb a concurrent ckv_select / ckv_select_decode of those problems: they
+ * read clusters [0, n_clusters) only, and the one shared entry,
+ * offsets[cluster_base], is rewritten with the value it holds
+ * (perm_base). Publishing the new clusters (raising n_clusters, moving
+ * tail_begin) is the caller's, after this call's work has completed.
+ * Errors as ckv_cluster, and CKV_ERR_INVALID for max_sms < 0. */
+ckv_status ckv_cluster_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                          int tok_begin, int tok_end, int C, int iters, int cluster_base,
+                          int perm_base, int C_cap, int perm_cap, float *centroids,
+                          void *centroids_hat, void *centroids_lp, int32_t *labels,
+                          int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
+                          size_t ws_bytes, int max_sms, void *stream);
+
 /* Stage: strided seeding only (mu, mu-hat and the scoring copy of clusters
  * [cluster_base, cluster_base + C)). Arguments as in ckv_cluster. */
 ckv_status ckv_init_centroids(const void *keys, ckv_dtype dt, int P, int64_t problem_stride,

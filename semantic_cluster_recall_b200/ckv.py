@@ -30,7 +30,7 @@ EXPORTS = [
     "ckv_select_workspace_bytes", "ckv_select",
     "ckv_decode_workspace_bytes", "ckv_sparse_decode", "ckv_append",
     "ckv_sparse_decode_noalloc_scratch_bytes", "ckv_sparse_decode_noalloc",
-    "ckv_select_decode",
+    "ckv_select_decode", "ckv_cluster_ex",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -70,6 +70,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "ckv_cluster_workspace_bytes": (sz, [i32, i32, i32]),
         "ckv_cluster": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32, i32, i32, i32,
                               vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ckv_cluster_ex": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32, i32, i32, i32,
+                                 vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, vp]),
         "ckv_init_centroids": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp]),
         "ckv_assign": (i32, [vp, i32, i32, i64, i32, i32, i32, vp, i32, i32, i32, vp, i32, i32,
@@ -160,6 +162,20 @@ def ckv_cluster(keys, problem_stride, tok_begin, tok_end, C, iters, cluster_base
                             _p(offsets), _p(perm), _p(ws), ws.numel() * ws.element_size(),
                             _stream(stream))
     _check(st, "ckv_cluster")
+
+
+def ckv_cluster_ex(keys, problem_stride, tok_begin, tok_end, C, iters, cluster_base, perm_base,
+                   C_cap, perm_cap, centroids, centroids_hat, centroids_lp, labels, sizes,
+                   offsets, perm, ws, max_sms=0, P=None, d=128, stream=None):
+    """ckv_cluster with the persistent assignment kernel held to max_sms SMs
+    (0 = all), for clustering in the background beside other GPU work."""
+    P = keys.shape[0] if P is None else P
+    st = load().ckv_cluster_ex(_p(keys), dtype_code(keys), P, problem_stride, d, tok_begin,
+                               tok_end, C, iters, cluster_base, perm_base, C_cap, perm_cap,
+                               _p(centroids), _p(centroids_hat), _p(centroids_lp), _p(labels),
+                               _p(sizes), _p(offsets), _p(perm), _p(ws),
+                               ws.numel() * ws.element_size(), int(max_sms), _stream(stream))
+    _check(st, "ckv_cluster_ex")
 
 
 def ckv_init_centroids(keys, problem_stride, tok_begin, tok_end, C, cluster_base, C_cap,

@@ -168,13 +168,15 @@ ckv_status launch_update(const T *keys, int P, int64_t pstride, int tok_begin, i
 
 ckv_status launch_assign(const void *keys, ckv_dtype dt, int P, int64_t pstride, int tok_begin,
                          int n, const void *hat, int C, int cbase, int C_cap, int32_t *labels,
-                         int perm_base, int perm_cap, cudaStream_t st) {
+                         int perm_base, int perm_cap, cudaStream_t st, int max_sms = 0) {
     if (dt == CKV_F32)
         return launch_assign_f32((const float *)keys, P, pstride, tok_begin, n, (const float *)hat,
                                  C, cbase, C_cap, labels, perm_base, perm_cap, st);
     ckv_status s = launch_assign_bf16((const bf16 *)keys, P, pstride, tok_begin, n,
                                       (const bf16 *)hat, C, cbase, C_cap, labels, perm_base,
-                                      perm_cap, sm_count(), st);
+                                      perm_cap,
+                                      max_sms > 0 && max_sms < sm_count() ? max_sms : sm_count(),
+                                      st);
     if (s) return fail(s, "tensor-core assignment launch failed (%s)",
                        cudaGetErrorString(cudaGetLastError()));
     return ok();
@@ -392,6 +394,19 @@ ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_st
                        void *centroids_hat, void *centroids_lp, int32_t *labels, int32_t *sizes,
                        int32_t *offsets, int32_t *perm, void *workspace, size_t ws_bytes,
                        void *stream) {
+    return ckv_cluster_ex(keys, dt, P, problem_stride, d, tok_begin, tok_end, C, iters,
+                          cluster_base, perm_base, C_cap, perm_cap, centroids, centroids_hat,
+                          centroids_lp, labels, sizes, offsets, perm, workspace, ws_bytes, 0,
+                          stream);
+}
+
+ckv_status ckv_cluster_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                          int tok_begin, int tok_end, int C, int iters, int cluster_base,
+                          int perm_base, int C_cap, int perm_cap, float *centroids,
+                          void *centroids_hat, void *centroids_lp, int32_t *labels,
+                          int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
+                          size_t ws_bytes, int max_sms, void *stream) {
+    if (max_sms < 0) return fail(CKV_ERR_INVALID, "max_sms must be >= 0 (got %d)", max_sms);
     ckv_status s = check_region(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
                                 cluster_base, C_cap);
     if (s) return s;
@@ -412,7 +427,7 @@ ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_st
         return s;
     for (int it = 0; it < iters; ++it) {
         if ((s = launch_assign(keys, dt, P, problem_stride, tok_begin, n, centroids_hat, C,
-                               cluster_base, C_cap, labels, perm_base, perm_cap, st)))
+                               cluster_base, C_cap, labels, perm_base, perm_cap, st, max_sms)))
             return s;
         if ((s = launch_index(labels, P, tok_begin, n, C, cluster_base, C_cap, perm_base, perm_cap,
                               offsets, perm, workspace, st)))

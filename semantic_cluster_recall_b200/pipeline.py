@@ -14,7 +14,13 @@ problems:
 * append(k, v) / incremental(): one generated token per step, and clustering
   of the oldest generated tokens into a few new clusters once the recent tail
   reaches its capacity ("III.B": generated tokens are clustered on their own
-  into four new centroids every so many steps).
+  into four new centroids every so many steps);
+* incremental_begin() / incremental_commit(): the same clustering started
+  early on a side stream, behind the decode steps of the main stream, and
+  published later ("IV.B Semantic Clustering": clustering is launched
+  asynchronously and overlaps other inference work). Until the commit the
+  steps read only the committed clusters; the new ones are written to
+  metadata slots no step reads.
 
 Nothing here computes: every step is one of libckv's kernels.
 """
@@ -63,6 +69,10 @@ class ClusterRecall:
         self.C_used = 0           # clusters used
         self.tail_lo = 0          # host copy of tail_begin (uniform over problems)
         self.scale = 1.0 / math.sqrt(d)
+        self._pending = None      # background clustering in flight: (n_tok, C, end, event)
+
+    def _main(self):
+        return self.stream if self.stream is not None else torch.cuda.current_stream(self.device)
 
     def _ws_cluster(self, n_tok: int, C: int) -> torch.Tensor:
         need = ckv.ckv_cluster_workspace_bytes(self.P, n_tok, C)
@@ -79,9 +89,10 @@ class ClusterRecall:
                         self.sizes, self.offsets, self.perm, ws, P=self.P, d=self.d,
                         stream=self.stream)
         self.n_clustered, self.C_used, self.tail_lo = te - tb, C, te
-        self.n_clusters.fill_(C)
-        self.tail_begin.fill_(te)
-        self.tail_end.fill_(L)
+        with torch.cuda.stream(self._main()):
+            self.n_clusters.fill_(C)
+            self.tail_begin.fill_(te)
+            self.tail_end.fill_(L)
 
     def incremental(self, K: torch.Tensor, n_tok: int, C: int, iters: int):
         """Cluster the oldest n_tok tail tokens into C new clusters appended to
@@ -95,8 +106,49 @@ class ClusterRecall:
         self.n_clustered += n_tok
         self.C_used += C
         self.tail_lo = te
-        self.n_clusters.fill_(self.C_used)
-        self.tail_begin.fill_(te)
+        with torch.cuda.stream(self._main()):
+            self.n_clusters.fill_(self.C_used)
+            self.tail_begin.fill_(te)
+
+    def incremental_begin(self, K: torch.Tensor, n_tok: int, C: int, iters: int,
+                          side_stream: torch.cuda.Stream, max_sms: int = 0):
+        """Start clustering the oldest n_tok tail tokens into C new clusters on
+        side_stream, after the work queued so far on the main stream (the
+        appends that wrote those tokens). The persistent assignment kernel is
+        held to max_sms SMs (0 = all), so that a low-priority side stream
+        leaves the rest of the GPU to the decode steps."""
+        if self._pending is not None:
+            raise RuntimeError("a background clustering is already in flight")
+        tb, te = self.tail_lo, self.tail_lo + n_tok
+        ws = self._ws_cluster(n_tok, C)
+        ws.record_stream(side_stream)
+        ready = torch.cuda.Event()
+        ready.record(self._main())
+        side_stream.wait_event(ready)
+        ckv.ckv_cluster_ex(K, K.stride(0), tb, te, C, iters, self.C_used, self.n_clustered,
+                           self.C_cap, self.perm_cap, self.centroids, self.centroids_hat,
+                           self.centroids_lp, self.labels, self.sizes, self.offsets, self.perm,
+                           ws, max_sms=max_sms, P=self.P, d=self.d, stream=side_stream)
+        done = torch.cuda.Event()
+        done.record(side_stream)
+        self._pending = (n_tok, C, te, done)
+
+    def incremental_commit(self):
+        """Publish the clusters of incremental_begin(): the main stream waits
+        for the side stream's work, then the steps see the new clusters and
+        the tail starts after their tokens."""
+        if self._pending is None:
+            raise RuntimeError("no background clustering in flight")
+        n_tok, C, te, done = self._pending
+        main = self._main()
+        main.wait_event(done)
+        self.n_clustered += n_tok
+        self.C_used += C
+        self.tail_lo = te
+        with torch.cuda.stream(main):
+            self.n_clusters.fill_(self.C_used)
+            self.tail_begin.fill_(te)
+        self._pending = None
 
     def select(self, q: torch.Tensor):
         ckv.ckv_select(q, self.centroids_lp, self.n_clusters, self.C_cap, self.offsets, self.perm,

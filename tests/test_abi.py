@@ -81,6 +81,13 @@ def test_validation_rejects_bad_arguments_without_launching(lib):
     # workspace too small
     _expect_invalid(lib.ckv_cluster(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 2, 0, 0, 8, 100,
                                     fake, fake, fake, fake, fake, fake, fake, fake, 16, None))
+    # background clustering: negative SM cap, and the same checks as ckv_cluster
+    _expect_invalid(lib.ckv_cluster_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 2, 0, 0, 8, 100,
+                                       fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
+                                       -1, None))
+    _expect_invalid(lib.ckv_cluster_ex(fake, 1, 2, 128 * 100, 128, 0, 3, 4, 2, 0, 0, 8, 100,
+                                       fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
+                                       16, None))
     # unknown dtype
     _expect_invalid(lib.ckv_assign(fake, 7, 2, 128 * 100, 128, 0, 100, fake, 4, 0, 8, fake, 0,
                                    100, None))
