@@ -25,6 +25,9 @@ import numpy as np
 from . import build as _build
 
 ROUND = {"none": 0, "f32": 1, "bf16": 2}
+# clustering similarity ("III.B": cosine, with L2 and inner product as the
+# paper's ablation)
+METRIC = {"cos": 0, "ip": 1, "l2": 2}
 
 _lib = None
 
@@ -52,6 +55,14 @@ def lib():
                                   f64p, f64p, i32p, i32p, i32p, i32p,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.ckvo_round.argtypes = [f64p, c_sz, c_int, f64p]
+        L.ckvo_init_m.argtypes = [f32p, c_int, c_int, c_int, c_int, c_int, f64p, f64p]
+        L.ckvo_assign_m.argtypes = [f32p, c_int, c_int, f64p, c_int, c_int, i32p,
+                                    ctypes.c_void_p]
+        L.ckvo_update_m.argtypes = [f32p, c_int, c_int, i32p, c_int, c_int, c_int, f64p, f64p,
+                                    i32p]
+        L.ckvo_kmeans_m.argtypes = [f32p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                    f64p, f64p, i32p, i32p, i32p, i32p,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.ckvo_score.argtypes = [f32p, c_int, c_int, f32p, c_int, f32p]
         L.ckvo_select.restype = c_int
         L.ckvo_select.argtypes = [f32p, c_int, i32p, i32p, c_int, c_int, i32p]
@@ -104,33 +115,46 @@ def round_to(x, mode: str) -> np.ndarray:
 
 # ---- clustering --------------------------------------------------------------
 
-def init(keys, C: int, mode: str):
+def init(keys, C: int, mode: str, metric: str = "cos"):
+    """Strided seeds mu and their assignment copy (mu/||mu|| for cosine, mu
+    for "ip" and "l2"), rounded to `mode`."""
     keys = _f32(keys)
     n, d = keys.shape
     mu = np.zeros((C, d), np.float64)
     muhat = np.zeros((C, d), np.float64)
-    lib().ckvo_init(keys, n, d, C, ROUND[mode], mu, muhat)
+    if metric == "cos":
+        lib().ckvo_init(keys, n, d, C, ROUND[mode], mu, muhat)
+    else:
+        lib().ckvo_init_m(keys, n, d, C, ROUND[mode], METRIC[metric], mu, muhat)
     return mu, muhat
 
 
-def assign(keys, muhat, with_gap: bool = True):
+def assign(keys, muhat, with_gap: bool = True, metric: str = "cos"):
     keys = _f32(keys)
     muhat = _f64(muhat)
     n, d = keys.shape
     labels = np.zeros(n, np.int32)
     gap = np.zeros(n, np.float64) if with_gap else None
-    lib().ckvo_assign(keys, n, d, muhat, muhat.shape[0], labels, _ptr(gap))
+    if metric == "cos":
+        lib().ckvo_assign(keys, n, d, muhat, muhat.shape[0], labels, _ptr(gap))
+    else:
+        lib().ckvo_assign_m(keys, n, d, muhat, muhat.shape[0], METRIC[metric], labels,
+                            _ptr(gap))
     return labels, gap
 
 
-def update(keys, labels, mu, muhat, mode: str):
+def update(keys, labels, mu, muhat, mode: str, metric: str = "cos"):
     keys = _f32(keys)
     mu = _f64(mu).copy()
     muhat = _f64(muhat).copy()
     n, d = keys.shape
     C = mu.shape[0]
     sizes = np.zeros(C, np.int32)
-    lib().ckvo_update(keys, n, d, _i32(labels), C, ROUND[mode], mu, muhat, sizes)
+    if metric == "cos":
+        lib().ckvo_update(keys, n, d, _i32(labels), C, ROUND[mode], mu, muhat, sizes)
+    else:
+        lib().ckvo_update_m(keys, n, d, _i32(labels), C, ROUND[mode], METRIC[metric], mu,
+                            muhat, sizes)
     return mu, muhat, sizes
 
 
@@ -144,7 +168,7 @@ def index(labels, C: int, tok_begin: int, perm_base: int = 0):
 
 
 def kmeans(keys, C: int, T: int, mode: str, tok_begin: int = 0, perm_base: int = 0,
-           history: bool = False) -> dict:
+           history: bool = False, metric: str = "cos") -> dict:
     """Strided init, T rounds of (assign, update), then the index (T >= 1)."""
     keys = _f32(keys)
     n, d = keys.shape
@@ -158,9 +182,14 @@ def kmeans(keys, C: int, T: int, mode: str, tok_begin: int = 0, perm_base: int =
         lh = r["labels_hist"] = np.zeros((T, n), np.int32)
         mh = r["muhat_hist"] = np.zeros((T + 1, C, d), np.float64)
         gh = r["gap_hist"] = np.zeros((T, n), np.float64)
-    lib().ckvo_kmeans(keys, n, d, C, T, ROUND[mode], tok_begin, perm_base, r["mu"], r["muhat"],
-                      r["labels"], r["sizes"], r["offsets"], r["perm"], _ptr(lh), _ptr(mh),
-                      _ptr(gh))
+    if metric == "cos":
+        lib().ckvo_kmeans(keys, n, d, C, T, ROUND[mode], tok_begin, perm_base, r["mu"],
+                          r["muhat"], r["labels"], r["sizes"], r["offsets"], r["perm"], _ptr(lh),
+                          _ptr(mh), _ptr(gh))
+    else:
+        lib().ckvo_kmeans_m(keys, n, d, C, T, ROUND[mode], METRIC[metric], tok_begin, perm_base,
+                            r["mu"], r["muhat"], r["labels"], r["sizes"], r["offsets"],
+                            r["perm"], _ptr(lh), _ptr(mh), _ptr(gh))
     return r
 
 
@@ -222,6 +251,6 @@ def map_problems(fn, items, threads: Optional[int] = None):
         return list(ex.map(fn, items))
 
 
-__all__ = ["ROUND", "lib", "bf16_bits", "bf16_value", "round_to", "init", "assign", "update",
+__all__ = ["ROUND", "METRIC", "lib", "bf16_bits", "bf16_value", "round_to", "init", "assign", "update",
            "index", "kmeans", "score", "select", "attended_rows", "attend", "map_problems",
            "threads_default"]

@@ -94,30 +94,61 @@ static void normalise_row(const double *mu, int d, int mode, double *muhat) {
 
 /* ---- clustering: "III.B Clustering in the Semantic Space" --------------- */
 
+/* Similarity: cosine (the method), with L2 and inner product as the paper's
+ * ablation of the clustering distance. */
+
+#define CKVO_METRIC_COSINE 0
+#define CKVO_METRIC_INNER 1
+#define CKVO_METRIC_L2 2
+
+/* The copy of a centroid that assignment compares keys with: mu/||mu|| for
+ * cosine, mu itself for inner product and L2, rounded to the storage format. */
+static void assign_copy(const double *mu, int d, int mode, int metric, double *out) {
+    if (metric == CKVO_METRIC_COSINE) {
+        normalise_row(mu, d, mode, out);
+        return;
+    }
+    for (int t = 0; t < d; ++t) out[t] = round_to(mu[t], mode);
+}
+
+/* Similarity of key k to assignment copy m; larger is closer. L2 uses the
+ * plain definition, minus half the squared distance. */
+static double similarity(const float *k, const double *m, int d, int metric) {
+    if (metric != CKVO_METRIC_L2) return dot_d(k, m, d);
+    double s = 0.0;
+    for (int t = 0; t < d; ++t) {
+        double e = (double)k[t] - m[t];
+        s += e * e;
+    }
+    return -0.5 * s;
+}
+
 /* Initial centroids. The paper does not say how k-means is seeded; this
  * build seeds deterministically by stride: centroid c starts at the key of
  * clustered offset c * floor(n / C). */
-void ckvo_init(const float *keys, int n, int d, int C, int mode, double *mu, double *muhat) {
+void ckvo_init_m(const float *keys, int n, int d, int C, int mode, int metric, double *mu,
+                 double *mhat) {
     int stride = n / C;
     for (int c = 0; c < C; ++c) {
         const float *k = keys + (size_t)c * stride * d;
         for (int t = 0; t < d; ++t) mu[(size_t)c * d + t] = (double)k[t];
-        normalise_row(mu + (size_t)c * d, d, mode, muhat + (size_t)c * d);
+        assign_copy(mu + (size_t)c * d, d, mode, metric, mhat + (size_t)c * d);
     }
 }
 
-/* Assignment: each key joins the centroid of highest cosine similarity. The
- * key's own norm does not change which centroid wins, so the score is
- * k_i . muhat_c; an exact tie goes to the lowest c. gap (optional) receives
- * (best - second best) / ||k_i||, the top-2 margin in cosine units. */
-void ckvo_assign(const float *keys, int n, int d, const double *muhat, int C,
-                 int32_t *labels, double *gap) {
+/* Assignment: each key joins the centroid of highest similarity; an exact
+ * tie goes to the lowest c. Under cosine the key's own norm does not change
+ * which centroid wins, so the score is k_i . muhat_c. gap (optional)
+ * receives (best - second best) / ||k_i||, the top-2 margin in cosine units
+ * under cosine. */
+void ckvo_assign_m(const float *keys, int n, int d, const double *mhat, int C, int metric,
+                   int32_t *labels, double *gap) {
     for (int i = 0; i < n; ++i) {
         const float *k = keys + (size_t)i * d;
         double best = -INFINITY, second = -INFINITY;
         int arg = 0;
         for (int c = 0; c < C; ++c) {
-            double s = dot_d(k, muhat + (size_t)c * d, d);
+            double s = similarity(k, mhat + (size_t)c * d, d, metric);
             if (s > best) {
                 second = best;
                 best = s;
@@ -137,11 +168,12 @@ void ckvo_assign(const float *keys, int n, int d, const double *muhat, int C,
     }
 }
 
-/* Update: each centroid becomes the mean of the raw keys assigned to it, and
- * muhat its normalised copy. A cluster with no keys, or whose mean is the zero
- * vector, keeps its previous mu and muhat. sizes receives the member counts. */
-void ckvo_update(const float *keys, int n, int d, const int32_t *labels, int C, int mode,
-                 double *mu, double *muhat, int32_t *sizes) {
+/* Update: each centroid becomes the mean of the raw keys assigned to it. A
+ * cluster with no keys keeps its previous mu and assignment copy; under
+ * cosine so does one whose mean is the zero vector (it has no direction).
+ * sizes receives the member counts. */
+void ckvo_update_m(const float *keys, int n, int d, const int32_t *labels, int C, int mode,
+                   int metric, double *mu, double *mhat, int32_t *sizes) {
     double *sum = (double *)calloc((size_t)C * d, sizeof(double));
     int32_t *cnt = (int32_t *)calloc((size_t)C, sizeof(int32_t));
     for (int i = 0; i < n; ++i) {
@@ -157,9 +189,9 @@ void ckvo_update(const float *keys, int n, int d, const int32_t *labels, int C, 
             double m = sum[(size_t)c * d + t] / (double)cnt[c];
             ss += m * m;
         }
-        if (ss == 0.0) continue;
+        if (metric == CKVO_METRIC_COSINE && ss == 0.0) continue;
         for (int t = 0; t < d; ++t) mu[(size_t)c * d + t] = sum[(size_t)c * d + t] / (double)cnt[c];
-        normalise_row(mu + (size_t)c * d, d, mode, muhat + (size_t)c * d);
+        assign_copy(mu + (size_t)c * d, d, mode, metric, mhat + (size_t)c * d);
     }
     free(sum);
     free(cnt);
@@ -183,22 +215,47 @@ void ckvo_index(const int32_t *labels, int n, int C, int tok_begin, int perm_bas
 }
 
 /* The whole clustering of one problem: strided init, then T rounds of
- * (assign, update), then the index of the final labels. Optional histories:
- * labels_hist [T][n] (labels of round t), muhat_hist [T+1][C][d] (the muhat
- * each round assigned with, plus the final one), gap_hist [T][n]. T >= 1. */
+ * (assign, update) under the given similarity, then the index of the final
+ * labels. Optional histories: labels_hist [T][n] (labels of round t),
+ * mhat_hist [T+1][C][d] (the assignment copy each round used, plus the final
+ * one), gap_hist [T][n]. T >= 1. */
+void ckvo_kmeans_m(const float *keys, int n, int d, int C, int T, int mode, int metric,
+                   int tok_begin, int perm_base, double *mu, double *mhat, int32_t *labels,
+                   int32_t *sizes, int32_t *offsets, int32_t *perm, int32_t *labels_hist,
+                   double *mhat_hist, double *gap_hist) {
+    ckvo_init_m(keys, n, d, C, mode, metric, mu, mhat);
+    for (int t = 0; t < T; ++t) {
+        if (mhat_hist) memcpy(mhat_hist + (size_t)t * C * d, mhat, sizeof(double) * (size_t)C * d);
+        ckvo_assign_m(keys, n, d, mhat, C, metric, labels,
+                      gap_hist ? gap_hist + (size_t)t * n : NULL);
+        if (labels_hist) memcpy(labels_hist + (size_t)t * n, labels, sizeof(int32_t) * (size_t)n);
+        ckvo_update_m(keys, n, d, labels, C, mode, metric, mu, mhat, sizes);
+    }
+    if (mhat_hist) memcpy(mhat_hist + (size_t)T * C * d, mhat, sizeof(double) * (size_t)C * d);
+    ckvo_index(labels, n, C, tok_begin, perm_base, offsets, perm);
+}
+
+/* The method's clustering (cosine similarity). */
+void ckvo_init(const float *keys, int n, int d, int C, int mode, double *mu, double *muhat) {
+    ckvo_init_m(keys, n, d, C, mode, CKVO_METRIC_COSINE, mu, muhat);
+}
+
+void ckvo_assign(const float *keys, int n, int d, const double *muhat, int C,
+                 int32_t *labels, double *gap) {
+    ckvo_assign_m(keys, n, d, muhat, C, CKVO_METRIC_COSINE, labels, gap);
+}
+
+void ckvo_update(const float *keys, int n, int d, const int32_t *labels, int C, int mode,
+                 double *mu, double *muhat, int32_t *sizes) {
+    ckvo_update_m(keys, n, d, labels, C, mode, CKVO_METRIC_COSINE, mu, muhat, sizes);
+}
+
 void ckvo_kmeans(const float *keys, int n, int d, int C, int T, int mode, int tok_begin,
                  int perm_base, double *mu, double *muhat, int32_t *labels, int32_t *sizes,
                  int32_t *offsets, int32_t *perm, int32_t *labels_hist, double *muhat_hist,
                  double *gap_hist) {
-    ckvo_init(keys, n, d, C, mode, mu, muhat);
-    for (int t = 0; t < T; ++t) {
-        if (muhat_hist) memcpy(muhat_hist + (size_t)t * C * d, muhat, sizeof(double) * (size_t)C * d);
-        ckvo_assign(keys, n, d, muhat, C, labels, gap_hist ? gap_hist + (size_t)t * n : NULL);
-        if (labels_hist) memcpy(labels_hist + (size_t)t * n, labels, sizeof(int32_t) * (size_t)n);
-        ckvo_update(keys, n, d, labels, C, mode, mu, muhat, sizes);
-    }
-    if (muhat_hist) memcpy(muhat_hist + (size_t)T * C * d, muhat, sizeof(double) * (size_t)C * d);
-    ckvo_index(labels, n, C, tok_begin, perm_base, offsets, perm);
+    ckvo_kmeans_m(keys, n, d, C, T, mode, CKVO_METRIC_COSINE, tok_begin, perm_base, mu, muhat,
+                  labels, sizes, offsets, perm, labels_hist, muhat_hist, gap_hist);
 }
 
 /* The copy of the centroids used for scoring: mu rounded to the storage

@@ -43,6 +43,15 @@ MUTANTS = [
     ("selection: ties to the higher cluster id", "return (x->c > y->c) - (x->c < y->c);",
      "return (x->c < y->c) - (x->c > y->c);"),
     ("attention: scale applied twice", "logit[j] = scale * s;", "logit[j] = scale * scale * s;"),
+    ("L2: distance with a plus sign", "double e = (double)k[t] - m[t];",
+     "double e = (double)k[t] + m[t];"),
+    ("L2: inner product used instead", "    if (metric != CKVO_METRIC_L2) return dot_d(k, m, d);",
+     "    return dot_d(k, m, d);"),
+    ("variants: assignment copy not rounded",
+     "for (int t = 0; t < d; ++t) out[t] = round_to(mu[t], mode);",
+     "for (int t = 0; t < d; ++t) out[t] = mu[t];"),
+    ("variants: zero mean kept under every similarity",
+     "if (metric == CKVO_METRIC_COSINE && ss == 0.0) continue;", "if (ss == 0.0) continue;"),
     ("attended set: recent window one token short", "for (int j = tail_begin; j < tail_end; ++j) rows[n++] = j;",
      "for (int j = tail_begin; j < tail_end - 1; ++j) rows[n++] = j;"),
 ]

@@ -366,3 +366,153 @@ def test_incremental_index_appends_after_prefill():
     assert pre["offsets"][-1] == 292 == inc["offsets"][0]
     assert inc["offsets"][-1] == 292 + 64
     assert sorted(inc["perm"].tolist()) == list(range(300, 364))
+
+
+# ---- similarity variants: L2 and inner product (the paper's ablation) -----------------------
+
+def _no_near_ties(gap, eps=1e-6):
+    return gap >= eps
+
+
+@pytest.mark.parametrize("n,C,d", [(300, 17, 16), (257, 40, 128)])
+def test_l2_assign_is_scipy_sqeuclidean_argmin(n, C, d):
+    from scipy.spatial.distance import cdist
+    rng = np.random.default_rng(n + C)
+    keys = rng.standard_normal((n, d)).astype(np.float32)
+    mu = rng.standard_normal((C, d)) * rng.uniform(0.2, 2.0, (C, 1))
+    lab, gap = oracle.assign(keys, mu, metric="l2")
+    ref = cdist(keys.astype(np.float64), mu, "sqeuclidean").argmin(axis=1)
+    ok = _no_near_ties(gap)
+    assert ok.mean() > 0.99
+    assert np.array_equal(lab[ok], ref[ok])
+    # the gap is half the squared-distance margin over ||k||
+    dist = cdist(keys.astype(np.float64), mu, "sqeuclidean")
+    srt = np.sort(dist, axis=1)
+    np.testing.assert_allclose(gap, 0.5 * (srt[:, 1] - srt[:, 0]) /
+                               np.linalg.norm(keys.astype(np.float64), axis=1), rtol=1e-9,
+                               atol=1e-12)
+
+
+def test_inner_product_assign_is_matmul_argmax_and_differs_from_cosine():
+    rng = np.random.default_rng(31)
+    n, C, d = 400, 24, 64
+    keys = rng.standard_normal((n, d)).astype(np.float32)
+    mu = rng.standard_normal((C, d)) * rng.uniform(0.1, 3.0, (C, 1))  # unequal norms
+    lab, gap = oracle.assign(keys, mu, metric="ip")
+    ref = np.argmax(keys.astype(np.float64) @ mu.T, axis=1)
+    ok = _no_near_ties(gap)
+    assert np.array_equal(lab[ok], ref[ok])
+    # with unequal centroid norms the inner product and the cosine disagree
+    unit = mu / np.linalg.norm(mu, axis=1, keepdims=True)
+    lab_cos, _ = oracle.assign(keys, unit)
+    assert (lab != lab_cos).mean() > 0.05
+
+
+def test_metric_cosine_entry_points_equal_the_cosine_functions():
+    rng = np.random.default_rng(5)
+    n, C, d = 500, 12, 128
+    keys = oracle.round_to(rng.standard_normal((n, d)), "bf16").astype(np.float32)
+    L = oracle.lib()
+    for mode in ("none", "bf16"):
+        mu, mh = oracle.init(keys, C, mode)
+        mu2, mh2 = np.zeros_like(mu), np.zeros_like(mh)
+        L.ckvo_init_m(keys, n, d, C, oracle.ROUND[mode], 0, mu2, mh2)
+        assert np.array_equal(mu, mu2) and np.array_equal(mh, mh2)
+        lab, gap = oracle.assign(keys, mh)
+        lab2 = np.zeros(n, np.int32)
+        gap2 = np.zeros(n)
+        L.ckvo_assign_m(keys, n, d, mh, C, 0, lab2, gap2.ctypes.data_as(oracle.ctypes.c_void_p))
+        assert np.array_equal(lab, lab2) and np.array_equal(gap, gap2)
+        r = oracle.update(keys, lab, mu, mh, mode)
+        mu3, mh3, sz3 = mu.copy(), mh.copy(), np.zeros(C, np.int32)
+        L.ckvo_update_m(keys, n, d, lab, C, oracle.ROUND[mode], 0, mu3, mh3, sz3)
+        assert np.array_equal(r[0], mu3) and np.array_equal(r[1], mh3)
+        assert np.array_equal(r[2], sz3)
+
+
+@pytest.mark.parametrize("metric", ["ip", "l2"])
+def test_variant_init_and_update_keep_the_raw_mean(metric):
+    rng = np.random.default_rng(8)
+    n, C, d = 103, 10, 128
+    keys = oracle.round_to(rng.standard_normal((n, d)), "bf16").astype(np.float32)
+    mu, mh = oracle.init(keys, C, "bf16", metric=metric)
+    stride = n // C
+    for c in range(C):
+        assert np.array_equal(mu[c], keys[c * stride].astype(np.float64))
+        assert np.array_equal(mh[c], mu[c])  # a bf16 key is its own rounding
+    lab = rng.integers(0, C - 1, n).astype(np.int32)  # cluster C-1 stays empty
+    lab[:3] = 0  # and cluster 0 is never empty
+    mu2, mh2, sz = oracle.update(keys, lab, mu, mh, "bf16", metric=metric)
+    kd = keys.astype(np.float64)
+    for c in range(C - 1):
+        m = kd[lab == c].mean(0)
+        np.testing.assert_allclose(mu2[c], m, rtol=1e-12, atol=1e-15)
+        assert np.array_equal(mh2[c], oracle.round_to(mu2[c], "bf16"))
+    assert sz[C - 1] == 0 and np.array_equal(mu2[C - 1], mu[C - 1])
+    assert np.array_equal(mh2[C - 1], mh[C - 1])
+
+
+def test_l2_lloyd_objective_is_monotone():
+    # J = sum_i ||k_i - mu_{a_i}||^2: assignment minimises it for fixed
+    # centroids and the mean minimises it for fixed labels
+    rng = np.random.default_rng(12)
+    n, C, d = 1500, 18, 24
+    keys = rng.standard_normal((n, d)).astype(np.float32)
+    r = oracle.kmeans(keys, C, 10, "none", history=True, metric="l2")
+    kd = keys.astype(np.float64)
+    J = []
+    for t in range(10):
+        lab = r["labels_hist"][t]
+        J.append(np.sum((kd - r["muhat_hist"][t][lab]) ** 2))
+        J.append(np.sum((kd - r["muhat_hist"][t + 1][lab]) ** 2))
+    assert np.all(np.diff(J) <= 1e-9 * abs(J[0]))
+    assert J[-1] < J[0]
+
+
+def test_l2_kmeans_fixed_point_equals_sklearn_lloyd():
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(21)
+    C, per, d = 8, 60, 16
+    centers = rng.standard_normal((C, d)) * 4.0
+    keys = (np.repeat(centers, per, axis=0) +
+            rng.standard_normal((C * per, d))).astype(np.float32)
+    keys = keys[rng.permutation(C * per)]
+    n = keys.shape[0]
+    r = oracle.kmeans(keys, C, 60, "none", metric="l2")
+    seeds = keys[np.arange(C) * (n // C)].astype(np.float64)
+    km = KMeans(n_clusters=C, init=seeds, n_init=1, max_iter=300, tol=0.0,
+                algorithm="lloyd").fit(keys.astype(np.float64))
+    assert np.array_equal(r["labels"], km.labels_)
+    np.testing.assert_allclose(r["mu"], km.cluster_centers_, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("metric", ["ip", "l2"])
+def test_variant_planted_partition_recovers_blocks(metric):
+    # blocks along distinct unit directions with one common norm: every
+    # similarity sends each key to its block's centroid
+    rng = np.random.default_rng(3)
+    C, per, d = 12, 20, 128
+    dirs = rng.standard_normal((C, d))
+    dirs /= np.linalg.norm(dirs, axis=1, keepdims=True)
+    keys = (np.repeat(dirs, per, axis=0) * 1.5).astype(np.float32)
+    r = oracle.kmeans(keys, C, 3, "none", history=True, metric=metric)
+    blocks = np.repeat(np.arange(C), per)
+    for t in range(3):
+        assert np.array_equal(r["labels_hist"][t], blocks)
+    np.testing.assert_allclose(r["mu"], keys[::per].astype(np.float64), rtol=1e-12)
+
+
+@pytest.mark.parametrize("metric", ["ip", "l2"])
+def test_variant_zero_mean_is_a_valid_centroid(metric):
+    # a cluster of k and -k has mean zero: without a direction it is kept
+    # under cosine, but it is an ordinary centroid for L2 and inner product
+    rng = np.random.default_rng(14)
+    d = 128
+    k = oracle.round_to(rng.standard_normal(d), "bf16")
+    keys = np.stack([k, -k, k * 2.0]).astype(np.float32)
+    lab = np.array([0, 0, 1], np.int32)
+    mu0 = rng.standard_normal((2, d))
+    mu, mh, sz = oracle.update(keys, lab, mu0, mu0, "bf16", metric=metric)
+    assert np.array_equal(mu[0], np.zeros(d)) and np.array_equal(mh[0], np.zeros(d))
+    mu_c, mh_c, _ = oracle.update(keys, lab, mu0, mu0, "bf16")
+    assert np.array_equal(mu_c[0], mu0[0])
