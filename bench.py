@@ -422,6 +422,43 @@ def incremental_overlap(w: synth.Workload, K, V, q, dev, n_steps: int = 8,
     return res
 
 
+def assign_variants(step: "Step", stream, pk, n: int = 10) -> dict:
+    """One assignment round of the bench workload under each similarity of the
+    paper's ablation (cosine, inner product, L2), seeded by each one's own
+    init; L2 adds an fp32 bias subtraction per score in the epilogue. CUDA
+    events, L2 flushed before each launch, median of n."""
+    w, K, dev = step.w, step.K, step.dev
+    tb, te = w.S, w.L - w.W
+    flops = 2.0 * w.N * w.C * w.d * w.P
+    cent = torch.zeros((w.P, w.C, w.d), device=dev)
+    hat = torch.zeros((w.P, w.C, w.d), dtype=w.torch_dtype, device=dev)
+    lp = torch.zeros_like(hat)
+    bias = torch.zeros((w.P, w.C), device=dev)
+    labels = torch.zeros((w.P, w.N), dtype=torch.int32, device=dev)
+    out = {}
+    for metric in ("cos", "ip", "l2"):
+        ckv.ckv_init_centroids_ex(K, K.stride(0), tb, te, w.C, 0, w.C, cent, hat, lp,
+                                  metric=metric, bias=bias, stream=stream)
+        b = bias if metric == "l2" else None
+        ts = []
+        for i in range(n + 2):
+            step.flush_l2()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ckv.ckv_assign_ex(K, K.stride(0), tb, te, hat, w.C, 0, w.C, labels, 0, w.N, bias=b,
+                              stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e-3)
+        t = statistics.median(ts)
+        out[metric] = {"us_per_round": t * 1e6, "tflops": flops / t / 1e12,
+                       "frac_of_peak": flops / t / 1e12 / pk["bf16_tflops"]}
+    del cent, hat, lp, bias, labels
+    return out
+
+
 def e2e_measure(w: synth.Workload, dev, stream, steps: int):
     """End to end through the public calls: pinned host K/V/q -> device, one
     ckv_cluster + ckv_select + ckv_sparse_decode, outputs -> pinned host."""
@@ -530,6 +567,7 @@ def run_ours(args):
         err = ckv.ckv_device_error()
         e2e_s, h2d, d2h = e2e_measure(w, dev, stream, max(2, min(args.steps, 3)))
         e2e_s = reduce_max(e2e_s, world, dev)
+        variants = assign_variants(step, stream, pk) if world == 1 else None
         del step
         torch.cuda.empty_cache()
         dec32 = None
@@ -588,6 +626,7 @@ def run_ours(args):
         "e2e": {"value": world * keys / e2e_s, "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
         "decode_32layer": dec32,
+        "assign_by_similarity": variants,
         "gpu_launches": launches,
         "device_error_flags": err,
     }

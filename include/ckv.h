@@ -89,6 +89,14 @@ typedef enum { CKV_F32 = 0, CKV_BF16 = 1 } ckv_dtype;
 #define CKV_DEVERR_OFFSETS 0x8u /* offsets not monotone or outside [0, perm_cap] */
 #define CKV_DEVERR_TIMEOUT 0x10u /* a bounded device wait gave up (the kernel stopped early) */
 
+/* Similarity that clustering assigns keys by ("III.B Clustering in the
+ * Semantic Space": cosine; the paper's ablation compares L2 and inner
+ * product). Inner product and L2 assign against the raw mean rounded to the
+ * storage type (centroids_hat holds that copy); L2 ranks by
+ * k . m - |m|^2 / 2 (the same argmin as |k - m|^2), with |m|^2 / 2 kept in
+ * an fp32 bias array. A zero mean is a valid centroid for both. */
+typedef enum { CKV_COSINE = 0, CKV_INNER = 1, CKV_L2 = 2 } ckv_metric;
+
 /* Largest supported number of clusters per problem (C_cap). */
 #define CKV_MAX_CLUSTERS 4096
 
@@ -109,6 +117,9 @@ ckv_status ckv_device_error(unsigned int *flags, int clear, void *stream);
  * n_tok = tok_end - tok_begin. */
 size_t ckv_index_workspace_bytes(int P, int n_tok, int C);
 size_t ckv_cluster_workspace_bytes(int P, int n_tok, int C);
+/* Workspace for ckv_cluster_ex: ckv_cluster_workspace_bytes plus, for L2, the
+ * bias of the clusters being built. 0 for an unknown metric. */
+size_t ckv_cluster_ex_workspace_bytes(int P, int n_tok, int C, int metric);
 
 /* Cosine k-means over the keys of [tok_begin, tok_end) of every problem
  * ("III.B Clustering in the Semantic Space": assign each key to the centroid
@@ -133,9 +144,12 @@ ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_st
                        int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
                        size_t ws_bytes, void *stream);
 
-/* ckv_cluster for background use beside other GPU work ("IV.B Semantic
- * Clustering": clustering is launched asynchronously and overlaps other
- * inference kernels). Identical arguments and results, plus
+/* ckv_cluster with a choice of similarity and for background use beside
+ * other GPU work ("IV.B Semantic Clustering": clustering is launched
+ * asynchronously and overlaps other inference kernels). Arguments as
+ * ckv_cluster, plus
+ *   metric    a ckv_metric (CKV_COSINE gives exactly ckv_cluster's results);
+ *             workspace >= ckv_cluster_ex_workspace_bytes(P, n_tok, C, metric)
  *   max_sms   upper bound on the SMs the persistent tensor-core assignment
  *             kernel occupies (0 = all); the other clustering kernels are
  *             short-lived CTAs that interleave with other streams' work, so
@@ -148,13 +162,14 @@ ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_st
  * offsets[cluster_base], is rewritten with the value it holds
  * (perm_base). Publishing the new clusters (raising n_clusters, moving
  * tail_begin) is the caller's, after this call's work has completed.
- * Errors as ckv_cluster, and CKV_ERR_INVALID for max_sms < 0. */
+ * Errors as ckv_cluster, and CKV_ERR_INVALID for an unknown metric or
+ * max_sms < 0. */
 ckv_status ckv_cluster_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
                           int tok_begin, int tok_end, int C, int iters, int cluster_base,
                           int perm_base, int C_cap, int perm_cap, float *centroids,
                           void *centroids_hat, void *centroids_lp, int32_t *labels,
                           int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
-                          size_t ws_bytes, int max_sms, void *stream);
+                          size_t ws_bytes, int metric, int max_sms, void *stream);
 
 /* Stage: strided seeding only (mu, mu-hat and the scoring copy of clusters
  * [cluster_base, cluster_base + C)). Arguments as in ckv_cluster. */
@@ -162,6 +177,13 @@ ckv_status ckv_init_centroids(const void *keys, ckv_dtype dt, int P, int64_t pro
                               int d, int tok_begin, int tok_end, int C, int cluster_base,
                               int C_cap, float *centroids, void *centroids_hat,
                               void *centroids_lp, void *stream);
+/* Seeding under a ckv_metric: centroids_hat = the seed key itself for
+ * CKV_INNER and CKV_L2; for CKV_L2 bias[p][cluster_base + c] (fp32, [P][C_cap],
+ * caller-owned) receives half its squared norm. bias may be null otherwise. */
+ckv_status ckv_init_centroids_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride,
+                                 int d, int tok_begin, int tok_end, int C, int cluster_base,
+                                 int C_cap, float *centroids, void *centroids_hat,
+                                 void *centroids_lp, int metric, float *bias, void *stream);
 
 /* Stage: assignment. labels[p][perm_base + i] = cluster_base + argmax_c
  * (k_i . centroids_hat[c]) over c in [0, C), ties to the lowest c. For bf16
@@ -171,6 +193,13 @@ ckv_status ckv_assign(const void *keys, ckv_dtype dt, int P, int64_t problem_str
                       int tok_begin, int tok_end, const void *centroids_hat, int C,
                       int cluster_base, int C_cap, int32_t *labels, int perm_base, int perm_cap,
                       void *stream);
+/* Assignment with a per-centroid bias: argmax_c (k_i . centroids_hat[c] -
+ * bias[p][cluster_base + c]) ([P][C_cap] fp32, as written by the _ex seeding
+ * and update for CKV_L2). A null bias is ckv_assign. */
+ckv_status ckv_assign_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                         int tok_begin, int tok_end, const void *centroids_hat, int C,
+                         int cluster_base, int C_cap, int32_t *labels, int perm_base,
+                         int perm_cap, const float *bias, void *stream);
 
 /* Stage: cluster index of the labels of slots [perm_base, perm_base + n_tok):
  * offsets[cluster_base + c] for c in [0, C] (the last one is
@@ -183,15 +212,26 @@ ckv_status ckv_index(const int32_t *labels, int P, int tok_begin, int tok_end, i
 
 /* Stage: centroid update from an index: for each cluster c in
  * [cluster_base, cluster_base + C), mu_c = mean of the keys at
- * perm[offsets[c] .. offsets[c+1]) (summed in fp32 in perm order), sizes[c] =
- * its member count, centroids_hat = mu/||mu|| and centroids_lp = mu, both
- * rounded to dtype. A cluster with no members or a zero mean keeps its
- * previous centroids. tok_begin/tok_end bound the valid perm entries. */
+ * perm[offsets[c] .. offsets[c+1]) (summed in double in perm order),
+ * sizes[c] = its member count, centroids_hat = mu/||mu|| and centroids_lp =
+ * mu, both rounded to dtype once from double. A cluster with no members or a
+ * zero mean keeps its previous centroids. tok_begin/tok_end bound the valid
+ * perm entries. */
 ckv_status ckv_update(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
                       int tok_begin, int tok_end, int C, int cluster_base, int C_cap,
                       const int32_t *offsets, const int32_t *perm, int perm_cap,
                       float *centroids, void *centroids_hat, void *centroids_lp,
                       int32_t *sizes, void *stream);
+/* Update under a ckv_metric: for CKV_INNER and CKV_L2 centroids_hat = mu
+ * rounded to dtype, a zero mean is kept as the centroid, and for CKV_L2
+ * bias[p][cluster_base + c] receives half the squared norm of that rounded
+ * copy (bias may be null otherwise). Clusters with no members keep their
+ * previous values, bias included. */
+ckv_status ckv_update_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                         int tok_begin, int tok_end, int C, int cluster_base, int C_cap,
+                         const int32_t *offsets, const int32_t *perm, int perm_cap,
+                         float *centroids, void *centroids_hat, void *centroids_lp,
+                         int32_t *sizes, int metric, float *bias, void *stream);
 
 /* ---- decode-time selection ---------------------------------------------- */
 

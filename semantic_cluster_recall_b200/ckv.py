@@ -30,7 +30,8 @@ EXPORTS = [
     "ckv_select_workspace_bytes", "ckv_select",
     "ckv_decode_workspace_bytes", "ckv_sparse_decode", "ckv_append",
     "ckv_sparse_decode_noalloc_scratch_bytes", "ckv_sparse_decode_noalloc",
-    "ckv_select_decode", "ckv_cluster_ex",
+    "ckv_select_decode", "ckv_cluster_ex", "ckv_cluster_ex_workspace_bytes",
+    "ckv_init_centroids_ex", "ckv_assign_ex", "ckv_update_ex",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -71,7 +72,14 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "ckv_cluster": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32, i32, i32, i32,
                               vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ckv_cluster_ex": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32, i32, i32, i32,
-                                 vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, vp]),
+                                 vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, i32, vp]),
+        "ckv_cluster_ex_workspace_bytes": (sz, [i32, i32, i32, i32]),
+        "ckv_init_centroids_ex": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32,
+                                        vp, vp, vp, i32, vp, vp]),
+        "ckv_assign_ex": (i32, [vp, i32, i32, i64, i32, i32, i32, vp, i32, i32, i32, vp, i32,
+                                i32, vp, vp]),
+        "ckv_update_ex": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32, vp, vp, i32,
+                                vp, vp, vp, vp, i32, vp, vp]),
         "ckv_init_centroids": (i32, [vp, i32, i32, i64, i32, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp]),
         "ckv_assign": (i32, [vp, i32, i32, i64, i32, i32, i32, vp, i32, i32, i32, vp, i32, i32,
@@ -164,18 +172,58 @@ def ckv_cluster(keys, problem_stride, tok_begin, tok_end, C, iters, cluster_base
     _check(st, "ckv_cluster")
 
 
+METRICS = {"cos": 0, "ip": 1, "l2": 2}  # ckv_metric: CKV_COSINE, CKV_INNER, CKV_L2
+
+
+def ckv_cluster_ex_workspace_bytes(P: int, n_tok: int, C: int, metric: str = "cos") -> int:
+    return int(load().ckv_cluster_ex_workspace_bytes(P, n_tok, C, METRICS[metric]))
+
+
 def ckv_cluster_ex(keys, problem_stride, tok_begin, tok_end, C, iters, cluster_base, perm_base,
                    C_cap, perm_cap, centroids, centroids_hat, centroids_lp, labels, sizes,
-                   offsets, perm, ws, max_sms=0, P=None, d=128, stream=None):
-    """ckv_cluster with the persistent assignment kernel held to max_sms SMs
-    (0 = all), for clustering in the background beside other GPU work."""
+                   offsets, perm, ws, metric="cos", max_sms=0, P=None, d=128, stream=None):
+    """ckv_cluster under a similarity ("cos", "ip", "l2"), with the persistent
+    assignment kernel held to max_sms SMs (0 = all) for clustering in the
+    background beside other GPU work."""
     P = keys.shape[0] if P is None else P
     st = load().ckv_cluster_ex(_p(keys), dtype_code(keys), P, problem_stride, d, tok_begin,
                                tok_end, C, iters, cluster_base, perm_base, C_cap, perm_cap,
                                _p(centroids), _p(centroids_hat), _p(centroids_lp), _p(labels),
                                _p(sizes), _p(offsets), _p(perm), _p(ws),
-                               ws.numel() * ws.element_size(), int(max_sms), _stream(stream))
+                               ws.numel() * ws.element_size(), METRICS[metric], int(max_sms),
+                               _stream(stream))
     _check(st, "ckv_cluster_ex")
+
+
+def ckv_init_centroids_ex(keys, problem_stride, tok_begin, tok_end, C, cluster_base, C_cap,
+                          centroids, centroids_hat, centroids_lp, metric="cos", bias=None,
+                          P=None, d=128, stream=None):
+    P = keys.shape[0] if P is None else P
+    st = load().ckv_init_centroids_ex(_p(keys), dtype_code(keys), P, problem_stride, d,
+                                      tok_begin, tok_end, C, cluster_base, C_cap, _p(centroids),
+                                      _p(centroids_hat), _p(centroids_lp), METRICS[metric],
+                                      _p(bias), _stream(stream))
+    _check(st, "ckv_init_centroids_ex")
+
+
+def ckv_assign_ex(keys, problem_stride, tok_begin, tok_end, centroids_hat, C, cluster_base,
+                  C_cap, labels, perm_base, perm_cap, bias=None, P=None, d=128, stream=None):
+    P = keys.shape[0] if P is None else P
+    st = load().ckv_assign_ex(_p(keys), dtype_code(keys), P, problem_stride, d, tok_begin,
+                              tok_end, _p(centroids_hat), C, cluster_base, C_cap, _p(labels),
+                              perm_base, perm_cap, _p(bias), _stream(stream))
+    _check(st, "ckv_assign_ex")
+
+
+def ckv_update_ex(keys, problem_stride, tok_begin, tok_end, C, cluster_base, C_cap, offsets,
+                  perm, perm_cap, centroids, centroids_hat, centroids_lp, sizes, metric="cos",
+                  bias=None, P=None, d=128, stream=None):
+    P = keys.shape[0] if P is None else P
+    st = load().ckv_update_ex(_p(keys), dtype_code(keys), P, problem_stride, d, tok_begin,
+                              tok_end, C, cluster_base, C_cap, _p(offsets), _p(perm), perm_cap,
+                              _p(centroids), _p(centroids_hat), _p(centroids_lp), _p(sizes),
+                              METRICS[metric], _p(bias), _stream(stream))
+    _check(st, "ckv_update_ex")
 
 
 def ckv_init_centroids(keys, problem_stride, tok_begin, tok_end, C, cluster_base, C_cap,

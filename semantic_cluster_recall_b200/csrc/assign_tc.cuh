@@ -71,6 +71,9 @@ struct Args {
     int total;           // tiles over all problems
     int nch, ch_rows;    // centroid chunks and rows per chunk (multiple of 16, <= 256)
     int32_t *labels;
+    const float *bias;   // problem p's cluster c at bias[p * bstride + c] (L2), or null
+    int bstride;
+    int bias_vec4;       // bias rows start 16-byte aligned
 };
 
 // ---- PTX wrappers ------------------------------------------------------------
@@ -213,7 +216,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 
 // ---- the kernel ----------------------------------------------------------------
 
-template <bool RESIDENT, int KST>
+// 16 consecutive bias values (L1-cached; every lane of a warp reads the same ones)
+__device__ __forceinline__ void load_bias16(const float *b, int vec4, float (&o)[16]) {
+    if (vec4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 t = __ldg(reinterpret_cast<const float4 *>(b) + q);
+            o[4 * q] = t.x;
+            o[4 * q + 1] = t.y;
+            o[4 * q + 2] = t.z;
+            o[4 * q + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] = __ldg(b + i);
+    }
+}
+
+// BIASM: 0 no bias; 1 bias read from global memory (L1); 2 bias cached per
+// epilogue warp in shared memory
+template <bool RESIDENT, int KST, int BIASM>
 __global__ void __launch_bounds__(NTHREADS, 1)
 k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmc,
             const Args a) {
@@ -240,6 +262,9 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     float *red_v = reinterpret_cast<float *>(bars + NBAR + 1);           // [2][PARTS-1][BM]
     int *red_i = reinterpret_cast<int *>(red_v + 2 * (EPI_PARTS - 1) * BM);
+    // per epilogue warp: the bias of its columns of every chunk, [nch][MAXG * 16]
+    float *wbias_all = reinterpret_cast<float *>(
+        (reinterpret_cast<uintptr_t>(red_i + 2 * (EPI_PARTS - 1) * BM) + 15) & ~uintptr_t(15));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -400,8 +425,22 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
         const int g_lo = min(ngroups, part * gper), g_hi = min(ngroups, g_lo + gper);
         int acc = 0, nt = 0;
         bool ok = true;
+        float *wbias = wbias_all + (size_t)warp * a.nch * (MAXG * 16);
+        int bias_p = -1;  // problem whose bias this warp holds
         for (int tile = t_begin; tile < t_end && ok; ++tile, ++nt) {
             const int p = tile / a.tpp, t = tile - p * a.tpp;
+            const float *bp = BIASM ? a.bias + (size_t)p * a.bstride : nullptr;
+            if (BIASM == 2 && p != bias_p) {  // this warp's columns, every chunk
+                __syncwarp();
+                for (int e = lane; e < a.nch * MAXG * 16; e += 32) {
+                    const int j = e / (MAXG * 16), r = e - j * (MAXG * 16);
+                    const int g = g_lo + r / 16, col = g * 16 + (r & 15);
+                    const int cc = j * a.ch_rows + col;
+                    wbias[e] = (g < g_hi && cc < a.C) ? __ldg(bp + cc) : 0.f;
+                }
+                __syncwarp();
+                bias_p = p;
+            }
             float best[CHAINS];
             int bidx[CHAINS];
 #pragma unroll
@@ -431,20 +470,45 @@ k_assign_tc(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUt
                 for (int u = 0; u < MAXG; ++u) {
                     const int gc = (g_lo + u) * 16;
                     if (g_lo + u < g_hi && gc < lim) {
+                        // L2: scores minus half the centroid's squared norm
+                        if (BIASM == 2) {  // from this warp's cached copy, 4 at a time
+                            const float4 *wb = reinterpret_cast<const float4 *>(
+                                wbias + j * (MAXG * 16) + u * 16);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 b4 = wb[q];
+                                v[u][4 * q] -= b4.x;
+                                v[u][4 * q + 1] -= b4.y;
+                                v[u][4 * q + 2] -= b4.z;
+                                v[u][4 * q + 3] -= b4.w;
+                            }
+                        }
+                        float bcol[16];
+                        if (BIASM == 1) {
+                            if (gc + 16 <= lim) {
+                                load_bias16(bp + c0 + gc, a.bias_vec4, bcol);
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    bcol[i] = gc + i < lim ? __ldg(bp + c0 + gc + i) : 0.f;
+                            }
+                        }
                         if (gc + 16 <= lim) {
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 const int k = (u * 16 + i) % CHAINS;
-                                const bool take = v[u][i] > best[k];
-                                best[k] = take ? v[u][i] : best[k];
+                                const float sc = BIASM == 1 ? v[u][i] - bcol[i] : v[u][i];
+                                const bool take = sc > best[k];
+                                best[k] = take ? sc : best[k];
                                 bidx[k] = take ? c0 + gc + i : bidx[k];
                             }
                         } else {
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 const int k = (u * 16 + i) % CHAINS;
-                                const bool take = (gc + i < lim) && v[u][i] > best[k];
-                                best[k] = take ? v[u][i] : best[k];
+                                const float sc = BIASM == 1 ? v[u][i] - bcol[i] : v[u][i];
+                                const bool take = (gc + i < lim) && sc > best[k];
+                                best[k] = take ? sc : best[k];
                                 bidx[k] = take ? c0 + gc + i : bidx[k];
                             }
                         }
@@ -572,7 +636,7 @@ inline TcPlan tc_plan(int C) {
 inline ckv_status launch_assign_bf16(const bf16 *keys, int P, int64_t pstride, int tok_begin,
                                      int n, const bf16 *hat, int C, int cbase, int C_cap,
                                      int32_t *labels, int perm_base, int perm_cap, int sms,
-                                     cudaStream_t st) {
+                                     const float *bias, int bstride, cudaStream_t st) {
     CUtensorMap mk, mc;
     const TcPlan pl = tc_plan(C);
     if (!make_map_bf16(&mk, keys, P, pstride / 128, pstride, tc::BM)) return CKV_ERR_CUDA;
@@ -590,19 +654,33 @@ inline ckv_status launch_assign_bf16(const bf16 *keys, int P, int64_t pstride, i
     a.nch = pl.nch;
     a.ch_rows = pl.ch_rows;
     a.labels = labels;
+    a.bias = bias;
+    a.bstride = bstride;
+    a.bias_vec4 = (bstride % 4 == 0 && ((uintptr_t)bias & 15) == 0) ? 1 : 0;
+    // L2: cache the bias per epilogue warp when shared memory allows
+    size_t smem = pl.smem;
+    const size_t bias_bytes = (size_t)tc::EPI_WARPS * pl.nch * tc::MAXG * 16 * sizeof(float) + 16;
+    const bool bias_smem = bias && pl.smem + bias_bytes <= (size_t)tc::SMEM_OPTIN_MAX;
+    if (bias_smem) smem += bias_bytes;
     const int grid = a.total < sms ? a.total : sms;
     cudaError_t e;
+#define CKV_TC_LAUNCH(RES, KS, BI)                                                        \
+    do {                                                                                  \
+        e = cudaFuncSetAttribute(tc::k_assign_tc<RES, KS, BI>,                            \
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+        if (e != cudaSuccess) return CKV_ERR_CUDA;                                        \
+        tc::k_assign_tc<RES, KS, BI><<<grid, tc::NTHREADS, smem, st>>>(mk, mc, a);        \
+    } while (0)
     if (pl.resident) {
-        e = cudaFuncSetAttribute(tc::k_assign_tc<true, 3>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
-        if (e != cudaSuccess) return CKV_ERR_CUDA;
-        tc::k_assign_tc<true, 3><<<grid, tc::NTHREADS, pl.smem, st>>>(mk, mc, a);
+        if (bias_smem) CKV_TC_LAUNCH(true, 3, 2);
+        else if (bias) CKV_TC_LAUNCH(true, 3, 1);
+        else CKV_TC_LAUNCH(true, 3, 0);
     } else {
-        e = cudaFuncSetAttribute(tc::k_assign_tc<false, 2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
-        if (e != cudaSuccess) return CKV_ERR_CUDA;
-        tc::k_assign_tc<false, 2><<<grid, tc::NTHREADS, pl.smem, st>>>(mk, mc, a);
+        if (bias_smem) CKV_TC_LAUNCH(false, 2, 2);
+        else if (bias) CKV_TC_LAUNCH(false, 2, 1);
+        else CKV_TC_LAUNCH(false, 2, 0);
     }
+#undef CKV_TC_LAUNCH
     return cudaGetLastError() == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }
 

@@ -85,6 +85,8 @@ enum { SLOT_ASSIGN_F32 = 0, SLOT_ASSIGN_BF16, SLOT_HIST, SLOT_SCATTER, SLOT_RANK
 
 bool valid_dtype(ckv_dtype dt) { return dt == CKV_F32 || dt == CKV_BF16; }
 
+bool valid_metric(int m) { return m == CKV_COSINE || m == CKV_INNER || m == CKV_L2; }
+
 int nchunks_of(int n) { return (n + IDX_CHUNK - 1) / IDX_CHUNK; }
 
 // common checks of a clustering region
@@ -118,20 +120,24 @@ ckv_status check_perm(int n, int perm_base, int perm_cap) {
 
 template <typename T>
 ckv_status launch_init(const T *keys, int P, int64_t pstride, int tok_begin, int n, int C,
-                       int cbase, int C_cap, float *cent, T *hat, T *lp, cudaStream_t st) {
+                       int cbase, int C_cap, float *cent, T *hat, T *lp, int metric, float *bias,
+                       int bstride, cudaStream_t st) {
     dim3 grid((C + 7) / 8, P);
-    k_init<T><<<grid, 256, 0, st>>>(keys, pstride, tok_begin, n, C, cbase, C_cap, cent, hat, lp);
+    k_init<T><<<grid, 256, 0, st>>>(keys, pstride, tok_begin, n, C, cbase, C_cap, cent, hat, lp,
+                                    metric, bias, bstride);
     return launched("k_init");
 }
 
 ckv_status launch_assign_f32(const float *keys, int P, int64_t pstride, int tok_begin, int n,
                              const float *hat, int C, int cbase, int C_cap, int32_t *labels,
-                             int perm_base, int perm_cap, cudaStream_t st) {
+                             int perm_base, int perm_cap, const float *bias, int bstride,
+                             cudaStream_t st) {
     cudaError_t e = smem_optin(k_assign_simt<float>, AS_SMEM, SLOT_ASSIGN_F32);
     if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "smem opt-in: %s", cudaGetErrorString(e));
     dim3 grid((n + AS_TILE - 1) / AS_TILE, P);
     k_assign_simt<float><<<grid, 256, AS_SMEM, st>>>(keys, pstride, tok_begin, n, hat, C, cbase,
-                                                     C_cap, labels, perm_base, perm_cap);
+                                                     C_cap, labels, perm_base, perm_cap, bias,
+                                                     bstride);
     return launched("k_assign_simt");
 }
 
@@ -158,25 +164,26 @@ ckv_status launch_index(const int32_t *labels, int P, int tok_begin, int n, int 
 template <typename T>
 ckv_status launch_update(const T *keys, int P, int64_t pstride, int tok_begin, int tok_end, int C,
                          int cbase, int C_cap, const int32_t *offsets, const int32_t *perm,
-                         int perm_cap, float *cent, T *hat, T *lp, int32_t *sizes,
-                         cudaStream_t st) {
+                         int perm_cap, float *cent, T *hat, T *lp, int32_t *sizes, int metric,
+                         float *bias, int bstride, cudaStream_t st) {
     dim3 grid((C + 7) / 8, P);
     k_update<T><<<grid, 256, 0, st>>>(keys, pstride, tok_begin, tok_end, C, cbase, C_cap, offsets,
-                                      perm, perm_cap, cent, hat, lp, sizes);
+                                      perm, perm_cap, cent, hat, lp, sizes, metric, bias, bstride);
     return launched("k_update");
 }
 
 ckv_status launch_assign(const void *keys, ckv_dtype dt, int P, int64_t pstride, int tok_begin,
                          int n, const void *hat, int C, int cbase, int C_cap, int32_t *labels,
-                         int perm_base, int perm_cap, cudaStream_t st, int max_sms = 0) {
+                         int perm_base, int perm_cap, cudaStream_t st, int max_sms,
+                         const float *bias, int bstride) {
     if (dt == CKV_F32)
         return launch_assign_f32((const float *)keys, P, pstride, tok_begin, n, (const float *)hat,
-                                 C, cbase, C_cap, labels, perm_base, perm_cap, st);
+                                 C, cbase, C_cap, labels, perm_base, perm_cap, bias, bstride, st);
     ckv_status s = launch_assign_bf16((const bf16 *)keys, P, pstride, tok_begin, n,
                                       (const bf16 *)hat, C, cbase, C_cap, labels, perm_base,
                                       perm_cap,
                                       max_sms > 0 && max_sms < sm_count() ? max_sms : sm_count(),
-                                      st);
+                                      bias, bstride, st);
     if (s) return fail(s, "tensor-core assignment launch failed (%s)",
                        cudaGetErrorString(cudaGetLastError()));
     return ok();
@@ -316,10 +323,25 @@ size_t ckv_cluster_workspace_bytes(int P, int n_tok, int C) {
     return ckv_index_workspace_bytes(P, n_tok, C);
 }
 
+size_t ckv_cluster_ex_workspace_bytes(int P, int n_tok, int C, int metric) {
+    const size_t w = ckv_index_workspace_bytes(P, n_tok, C);
+    if (w == 0 || !valid_metric(metric)) return 0;
+    return metric == CKV_L2 ? w + align256((size_t)P * C * sizeof(float)) : w;
+}
+
 ckv_status ckv_init_centroids(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
                               int tok_begin, int tok_end, int C, int cluster_base, int C_cap,
                               float *centroids, void *centroids_hat, void *centroids_lp,
                               void *stream) {
+    return ckv_init_centroids_ex(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
+                                 cluster_base, C_cap, centroids, centroids_hat, centroids_lp,
+                                 CKV_COSINE, nullptr, stream);
+}
+
+ckv_status ckv_init_centroids_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride,
+                                 int d, int tok_begin, int tok_end, int C, int cluster_base,
+                                 int C_cap, float *centroids, void *centroids_hat,
+                                 void *centroids_lp, int metric, float *bias, void *stream) {
     ckv_status s = check_region(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
                                 cluster_base, C_cap);
     if (s) return s;
@@ -327,18 +349,30 @@ ckv_status ckv_init_centroids(const void *keys, ckv_dtype dt, int P, int64_t pro
     if (n < C) return fail(CKV_ERR_INVALID, "fewer tokens (%d) than clusters (%d)", n, C);
     if (!centroids || !centroids_hat || !centroids_lp)
         return fail(CKV_ERR_INVALID, "null centroid array");
+    if (!valid_metric(metric)) return fail(CKV_ERR_INVALID, "unknown metric %d", metric);
+    if (metric == CKV_L2 && !bias) return fail(CKV_ERR_INVALID, "L2 needs the bias array");
+    float *b = metric == CKV_L2 ? bias + cluster_base : nullptr;
     if (dt == CKV_BF16)
         return launch_init((const bf16 *)keys, P, problem_stride, tok_begin, n, C, cluster_base,
-                           C_cap, centroids, (bf16 *)centroids_hat, (bf16 *)centroids_lp,
-                           S(stream));
+                           C_cap, centroids, (bf16 *)centroids_hat, (bf16 *)centroids_lp, metric,
+                           b, C_cap, S(stream));
     return launch_init((const float *)keys, P, problem_stride, tok_begin, n, C, cluster_base, C_cap,
-                       centroids, (float *)centroids_hat, (float *)centroids_lp, S(stream));
+                       centroids, (float *)centroids_hat, (float *)centroids_lp, metric, b, C_cap,
+                       S(stream));
 }
 
 ckv_status ckv_assign(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
                       int tok_begin, int tok_end, const void *centroids_hat, int C,
                       int cluster_base, int C_cap, int32_t *labels, int perm_base, int perm_cap,
                       void *stream) {
+    return ckv_assign_ex(keys, dt, P, problem_stride, d, tok_begin, tok_end, centroids_hat, C,
+                         cluster_base, C_cap, labels, perm_base, perm_cap, nullptr, stream);
+}
+
+ckv_status ckv_assign_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                         int tok_begin, int tok_end, const void *centroids_hat, int C,
+                         int cluster_base, int C_cap, int32_t *labels, int perm_base,
+                         int perm_cap, const float *bias, void *stream) {
     ckv_status s = check_region(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
                                 cluster_base, C_cap);
     if (s) return s;
@@ -346,8 +380,10 @@ ckv_status ckv_assign(const void *keys, ckv_dtype dt, int P, int64_t problem_str
     if (!centroids_hat || !labels) return fail(CKV_ERR_INVALID, "null centroids_hat or labels");
     if ((s = check_perm(n, perm_base, perm_cap))) return s;
     if (!aligned(centroids_hat, 16)) return fail(CKV_ERR_INVALID, "centroids_hat misaligned");
+    if (bias && !aligned(bias, 4)) return fail(CKV_ERR_INVALID, "bias misaligned");
     return launch_assign(keys, dt, P, problem_stride, tok_begin, n, centroids_hat, C, cluster_base,
-                         C_cap, labels, perm_base, perm_cap, S(stream));
+                         C_cap, labels, perm_base, perm_cap, S(stream), 0,
+                         bias ? bias + cluster_base : nullptr, C_cap);
 }
 
 ckv_status ckv_index(const int32_t *labels, int P, int tok_begin, int tok_end, int C,
@@ -373,19 +409,45 @@ ckv_status ckv_update(const void *keys, ckv_dtype dt, int P, int64_t problem_str
                       const int32_t *offsets, const int32_t *perm, int perm_cap,
                       float *centroids, void *centroids_hat, void *centroids_lp, int32_t *sizes,
                       void *stream) {
+    return ckv_update_ex(keys, dt, P, problem_stride, d, tok_begin, tok_end, C, cluster_base,
+                         C_cap, offsets, perm, perm_cap, centroids, centroids_hat, centroids_lp,
+                         sizes, CKV_COSINE, nullptr, stream);
+}
+
+namespace {
+ckv_status update_impl(const void *keys, ckv_dtype dt, int P, int64_t problem_stride,
+                       int tok_begin, int tok_end, int C, int cluster_base, int C_cap,
+                       const int32_t *offsets, const int32_t *perm, int perm_cap,
+                       float *centroids, void *centroids_hat, void *centroids_lp, int32_t *sizes,
+                       int metric, float *bias, int bstride, cudaStream_t st) {
+    if (dt == CKV_BF16)
+        return launch_update((const bf16 *)keys, P, problem_stride, tok_begin, tok_end, C,
+                             cluster_base, C_cap, offsets, perm, perm_cap, centroids,
+                             (bf16 *)centroids_hat, (bf16 *)centroids_lp, sizes, metric, bias,
+                             bstride, st);
+    return launch_update((const float *)keys, P, problem_stride, tok_begin, tok_end, C,
+                         cluster_base, C_cap, offsets, perm, perm_cap, centroids,
+                         (float *)centroids_hat, (float *)centroids_lp, sizes, metric, bias,
+                         bstride, st);
+}
+}  // namespace
+
+ckv_status ckv_update_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
+                         int tok_begin, int tok_end, int C, int cluster_base, int C_cap,
+                         const int32_t *offsets, const int32_t *perm, int perm_cap,
+                         float *centroids, void *centroids_hat, void *centroids_lp,
+                         int32_t *sizes, int metric, float *bias, void *stream) {
     ckv_status s = check_region(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
                                 cluster_base, C_cap);
     if (s) return s;
     if (!offsets || !perm || !centroids || !centroids_hat || !centroids_lp || !sizes)
         return fail(CKV_ERR_INVALID, "null pointer argument");
     if (perm_cap < 1) return fail(CKV_ERR_INVALID, "bad perm_cap %d", perm_cap);
-    if (dt == CKV_BF16)
-        return launch_update((const bf16 *)keys, P, problem_stride, tok_begin, tok_end, C,
-                             cluster_base, C_cap, offsets, perm, perm_cap, centroids,
-                             (bf16 *)centroids_hat, (bf16 *)centroids_lp, sizes, S(stream));
-    return launch_update((const float *)keys, P, problem_stride, tok_begin, tok_end, C,
-                         cluster_base, C_cap, offsets, perm, perm_cap, centroids,
-                         (float *)centroids_hat, (float *)centroids_lp, sizes, S(stream));
+    if (!valid_metric(metric)) return fail(CKV_ERR_INVALID, "unknown metric %d", metric);
+    if (metric == CKV_L2 && !bias) return fail(CKV_ERR_INVALID, "L2 needs the bias array");
+    return update_impl(keys, dt, P, problem_stride, tok_begin, tok_end, C, cluster_base, C_cap,
+                       offsets, perm, perm_cap, centroids, centroids_hat, centroids_lp, sizes,
+                       metric, metric == CKV_L2 ? bias + cluster_base : nullptr, C_cap, S(stream));
 }
 
 ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
@@ -396,8 +458,8 @@ ckv_status ckv_cluster(const void *keys, ckv_dtype dt, int P, int64_t problem_st
                        void *stream) {
     return ckv_cluster_ex(keys, dt, P, problem_stride, d, tok_begin, tok_end, C, iters,
                           cluster_base, perm_base, C_cap, perm_cap, centroids, centroids_hat,
-                          centroids_lp, labels, sizes, offsets, perm, workspace, ws_bytes, 0,
-                          stream);
+                          centroids_lp, labels, sizes, offsets, perm, workspace, ws_bytes,
+                          CKV_COSINE, 0, stream);
 }
 
 ckv_status ckv_cluster_ex(const void *keys, ckv_dtype dt, int P, int64_t problem_stride, int d,
@@ -405,8 +467,9 @@ ckv_status ckv_cluster_ex(const void *keys, ckv_dtype dt, int P, int64_t problem
                           int perm_base, int C_cap, int perm_cap, float *centroids,
                           void *centroids_hat, void *centroids_lp, int32_t *labels,
                           int32_t *sizes, int32_t *offsets, int32_t *perm, void *workspace,
-                          size_t ws_bytes, int max_sms, void *stream) {
+                          size_t ws_bytes, int metric, int max_sms, void *stream) {
     if (max_sms < 0) return fail(CKV_ERR_INVALID, "max_sms must be >= 0 (got %d)", max_sms);
+    if (!valid_metric(metric)) return fail(CKV_ERR_INVALID, "unknown metric %d", metric);
     ckv_status s = check_region(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
                                 cluster_base, C_cap);
     if (s) return s;
@@ -416,25 +479,37 @@ ckv_status ckv_cluster_ex(const void *keys, ckv_dtype dt, int P, int64_t problem
     if (!centroids || !centroids_hat || !centroids_lp || !labels || !sizes || !offsets || !perm)
         return fail(CKV_ERR_INVALID, "null output array");
     if ((s = check_perm(n, perm_base, perm_cap))) return s;
-    if (!workspace || ws_bytes < ckv_cluster_workspace_bytes(P, n, C) || !aligned(workspace, 256))
+    if (!workspace || ws_bytes < ckv_cluster_ex_workspace_bytes(P, n, C, metric) ||
+        !aligned(workspace, 256))
         return fail(CKV_ERR_INVALID, "workspace too small or not 256-byte aligned");
     if (!aligned(centroids_hat, 16) || !aligned(centroids_lp, 16) || !aligned(centroids, 16))
         return fail(CKV_ERR_INVALID, "centroid arrays must be 16-byte aligned");
     cudaStream_t st = S(stream);
-    if ((s = ckv_init_centroids(keys, dt, P, problem_stride, d, tok_begin, tok_end, C,
-                                cluster_base, C_cap, centroids, centroids_hat, centroids_lp,
-                                stream)))
-        return s;
+    // L2: half the squared norm of each assignment copy, [P][C] after the histograms
+    float *bias = metric == CKV_L2
+                      ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                  ckv_index_workspace_bytes(P, n, C))
+                      : nullptr;
+    if (dt == CKV_BF16)
+        s = launch_init((const bf16 *)keys, P, problem_stride, tok_begin, n, C, cluster_base, C_cap,
+                        centroids, (bf16 *)centroids_hat, (bf16 *)centroids_lp, metric, bias, C,
+                        st);
+    else
+        s = launch_init((const float *)keys, P, problem_stride, tok_begin, n, C, cluster_base,
+                        C_cap, centroids, (float *)centroids_hat, (float *)centroids_lp, metric,
+                        bias, C, st);
+    if (s) return s;
     for (int it = 0; it < iters; ++it) {
         if ((s = launch_assign(keys, dt, P, problem_stride, tok_begin, n, centroids_hat, C,
-                               cluster_base, C_cap, labels, perm_base, perm_cap, st, max_sms)))
+                               cluster_base, C_cap, labels, perm_base, perm_cap, st, max_sms, bias,
+                               C)))
             return s;
         if ((s = launch_index(labels, P, tok_begin, n, C, cluster_base, C_cap, perm_base, perm_cap,
                               offsets, perm, workspace, st)))
             return s;
-        if ((s = ckv_update(keys, dt, P, problem_stride, d, tok_begin, tok_end, C, cluster_base,
-                            C_cap, offsets, perm, perm_cap, centroids, centroids_hat,
-                            centroids_lp, sizes, stream)))
+        if ((s = update_impl(keys, dt, P, problem_stride, tok_begin, tok_end, C, cluster_base,
+                             C_cap, offsets, perm, perm_cap, centroids, centroids_hat,
+                             centroids_lp, sizes, metric, bias, C, st)))
             return s;
     }
     return ok();

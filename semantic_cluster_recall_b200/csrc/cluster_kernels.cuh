@@ -51,6 +51,22 @@ __device__ __forceinline__ void store4_rn<bf16>(bf16 *p, const double (&v)[4]) {
     *reinterpret_cast<uint2 *>(p) = u;
 }
 
+// the values store4_rn stores, as doubles
+template <typename T>
+__device__ __forceinline__ void round4_rn(const double (&v)[4], double (&r)[4]);
+
+template <>
+__device__ __forceinline__ void round4_rn<float>(const double (&v)[4], double (&r)[4]) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) r[t] = (double)(float)v[t];
+}
+
+template <>
+__device__ __forceinline__ void round4_rn<bf16>(const double (&v)[4], double (&r)[4]) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) r[t] = (double)__uint_as_float((uint32_t)bf16_bits_rn(v[t]) << 16);
+}
+
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
@@ -65,7 +81,8 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 template <typename T>
 __global__ void __launch_bounds__(256)
 k_init(const T *__restrict__ keys, int64_t pstride, int tok_begin, int n, int C, int cbase,
-       int C_cap, float *__restrict__ cent, T *__restrict__ hat, T *__restrict__ lp) {
+       int C_cap, float *__restrict__ cent, T *__restrict__ hat, T *__restrict__ lp, int metric,
+       float *__restrict__ bias, int bstride) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x * 8 + warp;
     const int p = blockIdx.y;
@@ -78,6 +95,14 @@ k_init(const T *__restrict__ keys, int64_t pstride, int tok_begin, int n, int C,
     const size_t o = ((size_t)p * C_cap + cbase + c) * D + lane * 4;
     store4(cent + o, v);
     store4(lp + o, v);
+    if (metric != CKV_COSINE) {  // the assignment copy is the key itself
+        store4(hat + o, v);
+        if (metric == CKV_L2) {
+            const double hb = 0.5 * ss;  // half the squared norm of the (exact) copy
+            if (lane == 0) bias[(size_t)p * bstride + c] = (float)hb;
+        }
+        return;
+    }
     double h[4] = {0.0, 0.0, 0.0, 0.0};
     if (ss > 0.0) {
         const double nrm = sqrt(ss);
@@ -101,7 +126,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 k_assign_simt(const T *__restrict__ keys, int64_t pstride, int tok_begin, int n,
               const T *__restrict__ hat, int C, int cbase, int C_cap,
-              int32_t *__restrict__ labels, int perm_base, int perm_cap) {
+              int32_t *__restrict__ labels, int perm_base, int perm_cap,
+              const float *__restrict__ bias, int bstride) {
     extern __shared__ __align__(16) float smf[];
     float *Ks = smf;                  // [D][64], channel-major
     float *Ms = smf + D * AS_TILE;    // [D][64]
@@ -162,12 +188,16 @@ k_assign_simt(const T *__restrict__ keys, int64_t pstride, int tok_begin, int n,
         for (int j = 0; j < 4; ++j) {
             const int c = c0 + tx * 4 + j;
             if (c < C) {
+                // L2: minus half the centroid's squared norm (k . m - |m|^2 / 2)
+                const float bj = bias ? bias[(size_t)p * bstride + c] : 0.f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (acc[i][j] > best[i]) {
-                        best[i] = acc[i][j];
+                for (int i = 0; i < 4; ++i) {
+                    const float sc = acc[i][j] - bj;
+                    if (sc > best[i]) {
+                        best[i] = sc;
                         bidx[i] = c;
                     }
+                }
             }
         }
     }
@@ -382,7 +412,8 @@ __global__ void __launch_bounds__(256)
 k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end, int C,
          int cbase, int C_cap, const int32_t *__restrict__ offsets,
          const int32_t *__restrict__ perm, int perm_cap, float *__restrict__ cent,
-         T *__restrict__ hat, T *__restrict__ lp, int32_t *__restrict__ sizes) {
+         T *__restrict__ hat, T *__restrict__ lp, int32_t *__restrict__ sizes, int metric,
+         float *__restrict__ bias, int bstride) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x * 8 + warp;
     const int p = blockIdx.y;
@@ -425,13 +456,26 @@ k_update(const T *__restrict__ keys, int64_t pstride, int tok_begin, int tok_end
     double mu[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) mu[t] = acc[t] / (double)n;
+    const size_t o = ((size_t)p * C_cap + cbase + c) * D + lane * 4;
+    if (metric != CKV_COSINE) {  // assignment copy = the mean rounded to storage
+        double r[4];
+        round4_rn<T>(mu, r);
+        store4_rn<float>(cent + o, mu);
+        store4_rn<T>(lp + o, mu);
+        store4_rn<T>(hat + o, mu);
+        if (metric == CKV_L2) {
+            const double hb =
+                0.5 * warp_sum_d(r[0] * r[0] + r[1] * r[1] + r[2] * r[2] + r[3] * r[3]);
+            if (lane == 0) bias[(size_t)p * bstride + c] = (float)hb;
+        }
+        return;
+    }
     const double ss = warp_sum_d(mu[0] * mu[0] + mu[1] * mu[1] + mu[2] * mu[2] + mu[3] * mu[3]);
     if (!(ss > 0.0)) return;
     const double nrm = sqrt(ss);
     double h[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) h[t] = mu[t] / nrm;
-    const size_t o = ((size_t)p * C_cap + cbase + c) * D + lane * 4;
     store4_rn<float>(cent + o, mu);
     store4_rn<T>(lp + o, mu);
     store4_rn<T>(hat + o, h);

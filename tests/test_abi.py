@@ -47,6 +47,12 @@ def test_status_strings(lib):
 def test_workspace_sizes(lib):
     assert ckv.ckv_cluster_workspace_bytes(32, 32688, 400) == 32 * 400 * 16 * 4
     assert ckv.ckv_cluster_workspace_bytes(0, 10, 10) == 0
+    # L2 adds the [P][C] fp32 bias, 256-byte aligned; the others need nothing more
+    base = ckv.ckv_cluster_workspace_bytes(32, 32688, 400)
+    assert ckv.ckv_cluster_ex_workspace_bytes(32, 32688, 400, "cos") == base
+    assert ckv.ckv_cluster_ex_workspace_bytes(32, 32688, 400, "ip") == base
+    assert ckv.ckv_cluster_ex_workspace_bytes(32, 32688, 400, "l2") == base + 32 * 400 * 4
+    assert ckv.load().ckv_cluster_ex_workspace_bytes(32, 32688, 400, 7) == 0
     assert ckv.ckv_select_workspace_bytes(32, 404) % 256 == 0
     assert ckv.ckv_decode_workspace_bytes(32, 1, 128, 1104) > 0
     assert ckv.ckv_decode_workspace_bytes(32, 1, 64, 1104) == 0
@@ -81,13 +87,28 @@ def test_validation_rejects_bad_arguments_without_launching(lib):
     # workspace too small
     _expect_invalid(lib.ckv_cluster(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 2, 0, 0, 8, 100,
                                     fake, fake, fake, fake, fake, fake, fake, fake, 16, None))
-    # background clustering: negative SM cap, and the same checks as ckv_cluster
+    # clustering with a similarity / in the background: unknown metric, negative
+    # SM cap, an L2 workspace without room for the bias, and ckv_cluster's checks
     _expect_invalid(lib.ckv_cluster_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 2, 0, 0, 8, 100,
                                        fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
-                                       -1, None))
+                                       3, 0, None))
+    _expect_invalid(lib.ckv_cluster_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 2, 0, 0, 8, 100,
+                                       fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
+                                       0, -1, None))
+    ws_cos = ckv.ckv_cluster_workspace_bytes(2, 100, 4)
+    _expect_invalid(lib.ckv_cluster_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 2, 0, 0, 8, 100,
+                                       fake, fake, fake, fake, fake, fake, fake, fake, ws_cos,
+                                       2, 0, None))
     _expect_invalid(lib.ckv_cluster_ex(fake, 1, 2, 128 * 100, 128, 0, 3, 4, 2, 0, 0, 8, 100,
                                        fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20,
-                                       16, None))
+                                       1, 16, None))
+    # stage calls with a similarity: unknown metric, L2 without a bias array
+    _expect_invalid(lib.ckv_init_centroids_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 0, 8,
+                                              fake, fake, fake, 5, fake, None))
+    _expect_invalid(lib.ckv_init_centroids_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 0, 8,
+                                              fake, fake, fake, 2, None, None))
+    _expect_invalid(lib.ckv_update_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 0, 8, fake, fake,
+                                      100, fake, fake, fake, fake, 2, None, None))
     # unknown dtype
     _expect_invalid(lib.ckv_assign(fake, 7, 2, 128 * 100, 128, 0, 100, fake, 4, 0, 8, fake, 0,
                                    100, None))
