@@ -66,6 +66,11 @@ def lib():
         L.ckvo_score.argtypes = [f32p, c_int, c_int, f32p, c_int, f32p]
         L.ckvo_select.restype = c_int
         L.ckvo_select.argtypes = [f32p, c_int, i32p, i32p, c_int, c_int, i32p]
+        L.ckvo_selected_clusters.restype = c_int
+        L.ckvo_selected_clusters.argtypes = [f32p, c_int, i32p, c_int, i32p, i32p]
+        L.ckvo_cache_step.restype = c_int
+        L.ckvo_cache_step.argtypes = [i32p, i32p, c_int, c_int, c_int, i32p, i32p,
+                                      ctypes.POINTER(ctypes.c_int32)]
         L.ckvo_attend.argtypes = [f32p, c_int, c_int, f32p, f32p, i32p, c_int, c_dbl, f64p]
         L.ckvo_attended_rows.restype = c_int
         L.ckvo_attended_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, i32p]
@@ -214,6 +219,37 @@ def select(s, offsets, perm, budget: int, perm_base: int = 0):
     return sel[:cnt].copy(), cnt
 
 
+# ---- the cache of selected clusters ("D. Caching KV of Selected Tokens") -------
+
+NEVER = -(1 << 30)  # last-selected step of a cluster that was never selected
+
+
+def selected_clusters(s, offsets, budget: int):
+    """The clusters a selection recalls, in rank order, and how many tokens of
+    each are recalled."""
+    s = _f32(s)
+    offsets = _i32(offsets)
+    C = s.size
+    clusters = np.zeros(max(C, 1), np.int32)
+    taken = np.zeros(max(C, 1), np.int32)
+    m = lib().ckvo_selected_clusters(s, C, offsets, budget, clusters, taken)
+    return clusters[:m].copy(), taken[:m].copy()
+
+
+def cache_step(clusters, taken, step: int, R: int, last: np.ndarray):
+    """One step of the cache of the last R steps' clusters; `last` (int32 [C],
+    NEVER for never-selected clusters) is updated in place. Returns (hits,
+    hit_tokens, misses in rank order)."""
+    clusters = _i32(clusters)
+    taken = _i32(taken)
+    assert last.dtype == np.int32 and last.flags["C_CONTIGUOUS"]
+    misses = np.zeros(max(clusters.size, 1), np.int32)
+    ht = ctypes.c_int32(0)
+    hits = lib().ckvo_cache_step(clusters, taken, clusters.size, step, R, last, misses,
+                                 ctypes.byref(ht))
+    return hits, int(ht.value), misses[:clusters.size - hits].copy()
+
+
 # ---- attention ---------------------------------------------------------------
 
 def attended_rows(sink: int, sel_idx, tail_begin: int, tail_end: int) -> np.ndarray:
@@ -252,5 +288,6 @@ def map_problems(fn, items, threads: Optional[int] = None):
 
 
 __all__ = ["ROUND", "METRIC", "lib", "bf16_bits", "bf16_value", "round_to", "init", "assign", "update",
-           "index", "kmeans", "score", "select", "attended_rows", "attend", "map_problems",
+           "index", "kmeans", "score", "select", "selected_clusters", "cache_step", "NEVER",
+           "attended_rows", "attend", "map_problems",
            "threads_default"]

@@ -344,6 +344,61 @@ int ckvo_select(const float *s, int C, const int32_t *offsets, const int32_t *pe
     return taken;
 }
 
+/* ---- caching the KV of selected clusters: "D. Caching KV of Selected
+ * Tokens" ---------------------------------------------------------------- */
+
+/* The clusters one selection recalls, in rank order: non-empty clusters
+ * walked from the highest score until the budget is met, as in ckvo_select.
+ * taken[j] receives how many tokens of clusters[j] are recalled (all of them
+ * except in a trimmed last cluster). Returns the number of clusters. */
+int ckvo_selected_clusters(const float *s, int C, const int32_t *offsets, int budget,
+                           int32_t *clusters, int32_t *taken) {
+    ranked_t *r = (ranked_t *)malloc(sizeof(ranked_t) * (size_t)(C > 0 ? C : 1));
+    for (int c = 0; c < C; ++c) {
+        r[c].s = s[c];
+        r[c].c = c;
+    }
+    qsort(r, (size_t)C, sizeof(ranked_t), rank_cmp);
+    int total = 0, m = 0;
+    for (int j = 0; j < C && total < budget; ++j) {
+        int c = r[j].c;
+        int n_c = offsets[c + 1] - offsets[c];
+        if (n_c == 0) continue;
+        int take = n_c <= budget - total ? n_c : budget - total;
+        clusters[m] = c;
+        taken[m] = take;
+        ++m;
+        total += take;
+    }
+    free(r);
+    return m;
+}
+
+/* One decoding step of a cache that keeps the clusters selected in the last R
+ * steps: cluster c is cached at `step` when it was selected at one of steps
+ * step - R .. step - 1 (last[c] holds the last step that selected it; a
+ * never-selected cluster holds a value far below any step). Counts the hits
+ * among this step's clusters and the recalled tokens of those hits, lists the
+ * misses (the clusters to load) in rank order, then records this step's
+ * selection in last. Returns the number of hits. */
+int ckvo_cache_step(const int32_t *clusters, const int32_t *taken, int n, int step, int R,
+                    int32_t *last, int32_t *misses, int32_t *hit_tokens) {
+    int hits = 0, nm = 0, ht = 0;
+    for (int j = 0; j < n; ++j) {
+        int c = clusters[j];
+        int cached = R > 0 && last[c] < step && last[c] >= step - R;
+        if (cached) {
+            hits += 1;
+            ht += taken[j];
+        } else {
+            misses[nm++] = c;
+        }
+    }
+    for (int j = 0; j < n; ++j) last[clusters[j]] = step;
+    *hit_tokens = ht;
+    return hits;
+}
+
 /* ---- attention: "II.A LLM Inference and KV Cache" ---------------------- */
 
 /* out[g] = sum_j softmax_j(scale * q_g . k_j) v_j over the rows listed in

@@ -52,6 +52,12 @@ MUTANTS = [
      "for (int t = 0; t < d; ++t) out[t] = mu[t];"),
     ("variants: zero mean kept under every similarity",
      "if (metric == CKVO_METRIC_COSINE && ss == 0.0) continue;", "if (ss == 0.0) continue;"),
+    ("cache: one step too long a window", "int cached = R > 0 && last[c] < step && last[c] >= step - R;",
+     "int cached = R > 0 && last[c] < step && last[c] >= step - R - 1;"),
+    ("cache: selection not recorded", "    for (int j = 0; j < n; ++j) last[clusters[j]] = step;",
+     "    for (int j = 0; j + 1 < n; ++j) last[clusters[j]] = step;"),
+    ("selected clusters: empty clusters listed", "        if (n_c == 0) continue;\n        int take",
+     "        int take"),
     ("attended set: recent window one token short", "for (int j = tail_begin; j < tail_end; ++j) rows[n++] = j;",
      "for (int j = tail_begin; j < tail_end - 1; ++j) rows[n++] = j;"),
 ]

@@ -516,3 +516,65 @@ def test_variant_zero_mean_is_a_valid_centroid(metric):
     assert np.array_equal(mu[0], np.zeros(d)) and np.array_equal(mh[0], np.zeros(d))
     mu_c, mh_c, _ = oracle.update(keys, lab, mu0, mu0, "bf16")
     assert np.array_equal(mu_c[0], mu0[0])
+
+
+# ---- the cache of the last R steps' clusters ("D. Caching KV of Selected Tokens") ----------
+
+@pytest.mark.parametrize("budget", [0, 1, 50, 400, 10_000])
+def test_selected_clusters_spell_out_the_token_selection(budget):
+    rng = np.random.default_rng(budget + 3)
+    C, n = 60, 2000
+    lab = rng.integers(0, C, n).astype(np.int32)
+    lab[lab == 7] = 8  # an empty cluster
+    offsets, perm = oracle.index(lab, C, 16)
+    s = rng.standard_normal(C).astype(np.float32)
+    s[10] = s[11]  # a score tie
+    sel, cnt = oracle.select(s, offsets, perm, budget)
+    cl, taken = oracle.selected_clusters(s, offsets, budget)
+    assert taken.sum() == cnt and np.all(taken > 0)
+    rebuilt = np.concatenate([perm[offsets[c]:offsets[c] + t] for c, t in zip(cl, taken)]
+                             or [np.zeros(0, np.int32)])
+    assert np.array_equal(rebuilt, sel)
+    sizes = np.diff(offsets)
+    assert np.all(taken[:-1] == sizes[cl[:-1]]) if cl.size else True
+    assert 7 not in cl
+
+
+def test_cache_step_matches_a_window_of_sets():
+    rng = np.random.default_rng(17)
+    C = 40
+    for R in (0, 1, 2, 5):
+        last = np.full(C, oracle.NEVER, np.int32)
+        history = []
+        for step in range(30):
+            m = int(rng.integers(1, 12))
+            cl = rng.choice(C, m, replace=False).astype(np.int32)
+            taken = rng.integers(1, 9, m).astype(np.int32)
+            hits, ht, misses = oracle.cache_step(cl, taken, step, R, last)
+            window = set().union(*history[-R:]) if R > 0 and history else set()
+            ref_hit = np.array([c in window for c in cl])
+            assert hits == ref_hit.sum() and ht == taken[ref_hit].sum()
+            assert np.array_equal(misses, cl[~ref_hit])  # rank order kept
+            history.append(set(cl.tolist()))
+            assert np.all(last[cl] == step)
+
+
+def test_cache_closed_forms():
+    C = 10
+    cl = np.array([3, 1, 4], np.int32)
+    taken = np.array([5, 5, 2], np.int32)
+    # the same selection every step: all hits from the second step on, for any R >= 1
+    last = np.full(C, oracle.NEVER, np.int32)
+    assert oracle.cache_step(cl, taken, 0, 1, last)[0] == 0
+    for step in range(1, 5):
+        hits, ht, misses = oracle.cache_step(cl, taken, step, 1, last)
+        assert hits == 3 and ht == 12 and misses.size == 0
+    # R = 0 keeps nothing
+    last = np.full(C, oracle.NEVER, np.int32)
+    for step in range(4):
+        assert oracle.cache_step(cl, taken, step, 0, last)[0] == 0
+    # a cluster selected R + 1 steps ago has left the cache
+    last = np.full(C, oracle.NEVER, np.int32)
+    oracle.cache_step(np.array([2], np.int32), np.array([4], np.int32), 0, 2, last)
+    assert oracle.cache_step(np.array([2], np.int32), np.array([4], np.int32), 3, 2, last)[0] == 0
+    assert oracle.cache_step(np.array([2], np.int32), np.array([4], np.int32), 5, 2, last)[0] == 1
