@@ -422,6 +422,32 @@ def incremental_overlap(w: synth.Workload, K, V, q, dev, n_steps: int = 8,
     return res
 
 
+def cache_hit_rates(step: "Step", stream, steps: int = 64, rhos=(0.9, 0.99), Rs=(1, 2)) -> dict:
+    """Hit rates of a cache of the clusters selected in the last R decode steps
+    ("D. Caching KV of Selected Tokens"; the paper reports 63% at R = 1 and
+    74% at R = 2 on real decoding) over `steps` fused steps of the bench
+    workload's own clustering, with queries that drift from step to step
+    (synth.correlated_queries, consecutive cosine ~ rho: a stand-in, since the
+    pages give no model of how decode queries evolve)."""
+    w, st = step.w, step.st
+    dirs = synth.directions_all(w, step.dev)
+    out = {"steps": steps}
+    for rho in rhos:
+        qs = synth.correlated_queries(w, dirs, steps, rho)
+        for R in Rs:
+            st.enable_cache(R)
+            acc = torch.zeros(4, dtype=torch.int64, device=step.dev)
+            for t in range(steps):
+                st.step(qs[t], step.K, step.V, step_no=t)
+                acc += st.cache_stats.sum(0)
+            h, n, ht, nt = (int(x) for x in acc.cpu())
+            out[f"rho{rho}_R{R}"] = {"cluster_hit_rate": h / max(n, 1),
+                                     "token_hit_rate": ht / max(nt, 1),
+                                     "clusters_per_step": n / steps / w.P}
+    st.cache_R = None
+    return out
+
+
 def assign_variants(step: "Step", stream, pk, n: int = 10) -> dict:
     """One assignment round of the bench workload under each similarity of the
     paper's ablation (cosine, inner product, L2), seeded by each one's own
@@ -568,6 +594,7 @@ def run_ours(args):
         e2e_s, h2d, d2h = e2e_measure(w, dev, stream, max(2, min(args.steps, 3)))
         e2e_s = reduce_max(e2e_s, world, dev)
         variants = assign_variants(step, stream, pk) if world == 1 else None
+        cache = cache_hit_rates(step, stream) if world == 1 else None
         del step
         torch.cuda.empty_cache()
         dec32 = None
@@ -627,6 +654,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
         "decode_32layer": dec32,
         "assign_by_similarity": variants,
+        "cluster_cache": cache,
         "gpu_launches": launches,
         "device_error_flags": err,
     }

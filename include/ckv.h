@@ -279,6 +279,34 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
                              const int32_t *tail_begin, const int32_t *tail_end, int max_tail,
                              float scale, float *out, void *stream);
 
+/* ckv_select_decode with the accounting of a cache that keeps the KV of the
+ * clusters selected in the last R decode steps ("D. Caching KV of Selected
+ * Tokens": the GPU cache retains the KV and cluster labels of the last R
+ * steps and loads only clusters absent from it; the paper settles on R = 1).
+ * Same selection and output, plus, per problem p:
+ *   last_sel     int32 [P][C_cap], caller-owned: the last step that selected
+ *                each cluster; initialise to a value far below any step (for
+ *                example -2^30); updated with this step's selection
+ *   step         this step's number (increasing from call to call)
+ *   R            steps the cache keeps (>= 0; 0 caches nothing)
+ *   cache_stats  int32 [P][4]: selected clusters that were cached (hits), the
+ *                selected (non-empty) clusters, recalled tokens of the hits,
+ *                recalled tokens (sel_cnt)
+ *   miss_list    int32 [P][C_cap] or null: the selected clusters that were not
+ *                cached (the ones to load), in rank order; its length is
+ *                cache_stats[1] - cache_stats[0]
+ * A null last_sel is ckv_select_decode. Errors as ckv_select_decode, and
+ * CKV_ERR_INVALID for a cache without cache_stats or with R < 0. */
+ckv_status ckv_select_decode_cached(const void *q, ckv_dtype dt, int P, int G, int d,
+                                    const void *centroids_lp, const int32_t *n_clusters,
+                                    int C_cap, const int32_t *offsets, const int32_t *perm,
+                                    int perm_cap, int budget, int32_t *sel_idx, int32_t *sel_cnt,
+                                    const void *K, const void *V, int64_t kv_problem_stride,
+                                    int kv_rows, int sink, const int32_t *tail_begin,
+                                    const int32_t *tail_end, int max_tail, float scale,
+                                    float *out, int32_t *last_sel, int step, int R,
+                                    int32_t *cache_stats, int32_t *miss_list, void *stream);
+
 /* ---- sparse decode attention -------------------------------------------- */
 
 /* max_rows bounds sink + budget + (tail_end - tail_begin) over all problems. */

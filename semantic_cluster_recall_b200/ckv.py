@@ -31,7 +31,7 @@ EXPORTS = [
     "ckv_decode_workspace_bytes", "ckv_sparse_decode", "ckv_append",
     "ckv_sparse_decode_noalloc_scratch_bytes", "ckv_sparse_decode_noalloc",
     "ckv_select_decode", "ckv_cluster_ex", "ckv_cluster_ex_workspace_bytes",
-    "ckv_init_centroids_ex", "ckv_assign_ex", "ckv_update_ex",
+    "ckv_init_centroids_ex", "ckv_assign_ex", "ckv_update_ex", "ckv_select_decode_cached",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -97,6 +97,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "ckv_sparse_decode_noalloc_scratch_bytes": (sz, [i32, i32, i32, i32]),
         "ckv_select_decode": (i32, [vp, i32, i32, i32, i32, vp, vp, i32, vp, vp, i32, i32, vp, vp,
                                     vp, vp, i64, i32, i32, vp, vp, i32, f32, vp, vp]),
+        "ckv_select_decode_cached": (i32, [vp, i32, i32, i32, i32, vp, vp, i32, vp, vp, i32, i32,
+                                           vp, vp, vp, vp, i64, i32, i32, vp, vp, i32, f32, vp,
+                                           vp, i32, i32, vp, vp, vp]),
         "ckv_sparse_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, vp,
                                             vp, i32, vp, vp, i32, f32, vp, vp]),
     }
@@ -284,6 +287,26 @@ def ckv_select_decode(q, centroids_lp, n_clusters, C_cap, offsets, perm, perm_ca
                                   kv_rows, sink, _p(tail_begin), _p(tail_end), max_tail,
                                   float(scale), _p(out), _stream(stream))
     _check(st, "ckv_select_decode")
+
+
+NEVER_SELECTED = -(1 << 30)  # last-selected step of a cluster no step selected
+
+
+def ckv_select_decode_cached(q, centroids_lp, n_clusters, C_cap, offsets, perm, perm_cap, budget,
+                             sel_idx, sel_cnt, K, V, kv_problem_stride, kv_rows, sink, tail_begin,
+                             tail_end, max_tail, scale, out, last_sel, step, R, cache_stats,
+                             miss_list=None, P=None, G=None, d=128, stream=None):
+    """ckv_select_decode plus the accounting of a cache of the clusters
+    selected in the last R steps (last_sel: int32 [P][C_cap], initialised to
+    NEVER_SELECTED; cache_stats: int32 [P][4])."""
+    P = q.shape[0] if P is None else P
+    G = q.shape[1] if G is None else G
+    st = load().ckv_select_decode_cached(
+        _p(q), dtype_code(q), P, G, d, _p(centroids_lp), _p(n_clusters), C_cap, _p(offsets),
+        _p(perm), perm_cap, budget, _p(sel_idx), _p(sel_cnt), _p(K), _p(V), kv_problem_stride,
+        kv_rows, sink, _p(tail_begin), _p(tail_end), max_tail, float(scale), _p(out),
+        _p(last_sel), int(step), int(R), _p(cache_stats), _p(miss_list), _stream(stream))
+    _check(st, "ckv_select_decode_cached")
 
 
 def ckv_sparse_decode(q, K, V, kv_problem_stride, kv_rows, sink, tail_begin, tail_end, max_tail,

@@ -577,6 +577,24 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
                              const void *V, int64_t kv_problem_stride, int kv_rows, int sink,
                              const int32_t *tail_begin, const int32_t *tail_end, int max_tail,
                              float scale, float *out, void *stream) {
+    return ckv_select_decode_cached(q, dt, P, G, d, centroids_lp, n_clusters, C_cap, offsets,
+                                    perm, perm_cap, budget, sel_idx, sel_cnt, K, V,
+                                    kv_problem_stride, kv_rows, sink, tail_begin, tail_end,
+                                    max_tail, scale, out, nullptr, 0, 0, nullptr, nullptr,
+                                    stream);
+}
+
+ckv_status ckv_select_decode_cached(const void *q, ckv_dtype dt, int P, int G, int d,
+                                    const void *centroids_lp, const int32_t *n_clusters,
+                                    int C_cap, const int32_t *offsets, const int32_t *perm,
+                                    int perm_cap, int budget, int32_t *sel_idx, int32_t *sel_cnt,
+                                    const void *K, const void *V, int64_t kv_problem_stride,
+                                    int kv_rows, int sink, const int32_t *tail_begin,
+                                    const int32_t *tail_end, int max_tail, float scale,
+                                    float *out, int32_t *last_sel, int step, int R,
+                                    int32_t *cache_stats, int32_t *miss_list, void *stream) {
+    if (last_sel && (!cache_stats || R < 0))
+        return fail(CKV_ERR_INVALID, "a cache needs cache_stats and R >= 0");
     if (!q || !centroids_lp || !n_clusters || !offsets || !perm || !sel_cnt || !K || !V ||
         !tail_begin || !tail_end || !out)
         return fail(CKV_ERR_INVALID, "null pointer argument");
@@ -663,6 +681,11 @@ ckv_status ckv_select_decode(const void *q, ckv_dtype dt, int P, int G, int d,
     a.sel_idx = sel_idx;
     a.sel_cnt = sel_cnt;
     a.out = out;
+    a.last_sel = last_sel;
+    a.step = step;
+    a.R = R;
+    a.cache_stats = cache_stats;
+    a.miss_list = miss_list;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nc, P, 1);
     cfg.blockDim = dim3(sd::THREADS, 1, 1);

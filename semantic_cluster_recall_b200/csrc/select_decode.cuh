@@ -72,6 +72,11 @@ struct Args {
     int32_t *sel_idx;
     int32_t *sel_cnt;
     float *out;
+    // cache of the clusters selected in the last R steps (null: no cache)
+    int32_t *last_sel;     // [P][C_cap] last step that selected each cluster
+    int step, R;
+    int32_t *cache_stats;  // [P][4] hits, selected clusters, hit tokens, recalled tokens
+    int32_t *miss_list;    // [P][C_cap] selected clusters not cached, rank order (or null)
 };
 
 // dynamic shared memory layout (bytes), sized by C_cap, G and chunk
@@ -125,6 +130,7 @@ k_select_decode(const Args a) {
     __shared__ __align__(16) unsigned s_hw[2][256];  // size sum per digit
     __shared__ __align__(16) unsigned s_hn[2][256];  // cluster count per digit
     __shared__ int s_before, s_total, s_bin, s_cnt, s_m;
+    __shared__ int s_wm[WARPS], s_hits, s_htok;
 
     const int nC = min(max(a.ncl[p], 0), a.C_cap);
     const int32_t *off = a.offsets + (size_t)p * (a.C_cap + 1);
@@ -314,6 +320,59 @@ k_select_decode(const Args a) {
         start[r] = st;
     }
     __syncthreads();
+
+    // ---- cache accounting ("D. Caching KV of Selected Tokens"): a selected
+    // cluster is a hit when one of the last R steps selected it; misses (the
+    // clusters a tiered cache would load) are listed in rank order; then this
+    // step is recorded. CTA 0 of the problem, thread per selected cluster ----
+    if (a.last_sel && rank == 0) {  // CTA-uniform
+        if (tid == 0) {
+            s_hits = 0;
+            s_htok = 0;
+        }
+        __syncthreads();
+        int32_t *last = a.last_sel + (size_t)p * a.C_cap;
+        int mbase = 0;
+        for (int r0 = 0; r0 < nsel; r0 += THREADS) {
+            const int r = r0 + tid;
+            int c = -1;
+            bool hit = false;
+            int tk = 0;
+            if (r < nsel) {
+                c = order[r];
+                tk = min(csz[c], cnt - start[r]);
+                const int l = last[c];
+                hit = a.R > 0 && l < a.step && l >= a.step - a.R;
+                last[c] = a.step;
+            }
+            const unsigned miss = __ballot_sync(FULL, r < nsel && !hit);
+            const int wh = __reduce_add_sync(FULL, hit ? 1 : 0);
+            const int wt = __reduce_add_sync(FULL, hit ? tk : 0);
+            if (lane == 0) {
+                s_wm[warp] = __popc(miss);
+                atomicAdd(&s_hits, wh);
+                atomicAdd(&s_htok, wt);
+            }
+            __syncthreads();
+            int wpre = 0, tot = 0;
+#pragma unroll
+            for (int w2 = 0; w2 < WARPS; ++w2) {
+                wpre += w2 < warp ? s_wm[w2] : 0;
+                tot += s_wm[w2];
+            }
+            if (a.miss_list && r < nsel && !hit)
+                a.miss_list[(size_t)p * a.C_cap + mbase + wpre + __popc(miss & lanemask_lt())] = c;
+            mbase += tot;
+            __syncthreads();
+        }
+        if (tid == 0) {
+            int32_t *cs = a.cache_stats + (size_t)p * 4;
+            cs[0] = s_hits;
+            cs[1] = nsel;
+            cs[2] = s_htok;
+            cs[3] = cnt;
+        }
+    }
 
     // ---- 4. resolve this CTA's rows of the attended list ----
     const int tb = a.tail_b[p];

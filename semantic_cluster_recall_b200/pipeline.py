@@ -70,6 +70,7 @@ class ClusterRecall:
         self.tail_lo = 0          # host copy of tail_begin (uniform over problems)
         self.scale = 1.0 / math.sqrt(d)
         self._pending = None      # background clustering in flight: (n_tok, C, end, event)
+        self.cache_R: Optional[int] = None  # cache of the last R steps' clusters, if enabled
 
     def _main(self):
         return self.stream if self.stream is not None else torch.cuda.current_stream(self.device)
@@ -162,9 +163,34 @@ class ClusterRecall:
                               d=self.d, stream=self.stream)
         return self.out
 
-    def step(self, q, K, V) -> torch.Tensor:
+    def enable_cache(self, R: int):
+        """Account a cache of the clusters selected in the last R steps ("D.
+        Caching KV of Selected Tokens"): every later step(..., step_no=t)
+        records per problem the hits, the selected clusters, the recalled
+        tokens of the hits and all recalled tokens in cache_stats, and the
+        clusters to load in miss_list."""
+        P, dev = self.P, self.device
+        self.cache_R = int(R)
+        self.last_sel = torch.full((P, self.C_cap), ckv.NEVER_SELECTED, dtype=torch.int32,
+                                   device=dev)
+        self.cache_stats = torch.zeros((P, 4), dtype=torch.int32, device=dev)
+        self.miss_list = torch.zeros((P, self.C_cap), dtype=torch.int32, device=dev)
+
+    def step(self, q, K, V, step_no: Optional[int] = None) -> torch.Tensor:
         """One decode step: selection then sparse attention, as one fused
-        launch (ckv_select_decode) when the shape allows it."""
+        launch (ckv_select_decode) when the shape allows it; with the cache
+        enabled, also its accounting for step number step_no."""
+        if self.cache_R is not None:
+            if step_no is None or self.G not in (1, 2, 4):
+                raise ValueError("a cached step needs step_no and G in (1, 2, 4)")
+            ckv.ckv_select_decode_cached(q, self.centroids_lp, self.n_clusters, self.C_cap,
+                                         self.offsets, self.perm, self.perm_cap, self.B,
+                                         self.sel_idx, self.sel_cnt, K, V, K.stride(0),
+                                         self.kv_rows, self.S, self.tail_begin, self.tail_end,
+                                         self.max_tail, self.scale, self.out, self.last_sel,
+                                         step_no, self.cache_R, self.cache_stats, self.miss_list,
+                                         P=self.P, G=self.G, d=self.d, stream=self.stream)
+            return self.out
         if self.G in (1, 2, 4):
             ckv.ckv_select_decode(q, self.centroids_lp, self.n_clusters, self.C_cap,
                                   self.offsets, self.perm, self.perm_cap, self.B, self.sel_idx,

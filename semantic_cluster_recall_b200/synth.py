@@ -208,6 +208,27 @@ def make_queries_batched(w: Workload, dirs: torch.Tensor, step: int) -> torch.Te
     return mixture_rows(dirs, w.G, w.sigma, g, scale=w.q_scale).to(w.torch_dtype)
 
 
+def correlated_queries(w: Workload, dirs: torch.Tensor, steps: int, rho: float) -> torch.Tensor:
+    """A sequence of decode queries [steps, P, G, d] whose direction drifts:
+    q_t = |q_{t-1}| * normalise(rho * u_{t-1} + sqrt(1 - rho^2) * e_t), with
+    u_{t-1} = q_{t-1} / |q_{t-1}| and e_t the unit direction of a fresh mixture
+    query (make_queries_batched), q_0 a fresh query. rho = 0 gives independent
+    steps; rho -> 1 repeats the first query. Consecutive decode queries of a
+    language model are correlated; the pages give no model of it, so this is a
+    stand-in whose rho is a free parameter."""
+    out = torch.empty((steps,) + tuple(dirs.shape[:1]) + (w.G, w.d), dtype=w.torch_dtype,
+                      device=dirs.device)
+    q = make_queries_batched(w, dirs, 0).float()
+    out[0] = q.to(w.torch_dtype)
+    a, b = float(rho), float((1.0 - rho * rho) ** 0.5)
+    for t in range(1, steps):
+        e = _unit_rows(make_queries_batched(w, dirs, t).float())
+        nrm = torch.linalg.vector_norm(q, dim=-1, keepdim=True)
+        q = nrm * _unit_rows(a * _unit_rows(q) + b * e)
+        out[t] = q.to(w.torch_dtype)
+    return out
+
+
 def random_labels(P: int, n: int, C: int, seed: int, device="cpu",
                   skew: float = 0.0) -> torch.Tensor:
     """Seeded cluster labels [P, n] int32 in [0, C), for stage-level tests.

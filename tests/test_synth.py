@@ -54,3 +54,19 @@ def test_random_labels_range_and_skew():
     assert lab.min() >= 0 and lab.max() < 50
     cnt = np.bincount(lab[0], minlength=50)
     assert cnt[0] > cnt[-1]
+
+
+def test_correlated_queries_drift_with_rho():
+    w = synth.WORKLOADS["llama2_layer_32k"].replace(P=4, L=256)
+    dirs = synth.directions_all(w, "cpu")
+    for rho in (0.0, 0.9, 0.99):
+        q = synth.correlated_queries(w, dirs, 6, rho).float()
+        assert q.shape == (6, 4, 1, 128)
+        cos = torch.nn.functional.cosine_similarity(q[1:], q[:-1], dim=-1)
+        assert abs(cos.mean().item() - rho) < 0.05
+        # norms carry over from the first query
+        n = torch.linalg.vector_norm(q, dim=-1)
+        assert torch.allclose(n, n[:1].expand_as(n), rtol=2e-2)
+    q1 = synth.correlated_queries(w, dirs, 3, 0.5)
+    q2 = synth.correlated_queries(w, dirs, 3, 0.5)
+    assert torch.equal(q1, q2)
