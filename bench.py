@@ -486,8 +486,11 @@ def assign_variants(step: "Step", stream, pk, n: int = 10) -> dict:
 
 
 def e2e_measure(w: synth.Workload, dev, stream, steps: int):
-    """End to end through the public calls: pinned host K/V/q -> device, one
-    ckv_cluster + ckv_select + ckv_sparse_decode, outputs -> pinned host."""
+    """End to end through the public calls: pinned host K/V/q -> device, the
+    clustering (ckv_cluster per group of problems, each group starting as soon
+    as its keys have arrived: ClusterRecall.prefill_from_host overlaps the
+    upload, the bound here, with the clustering), one fused decode step,
+    outputs -> pinned host."""
     Kh = torch.empty((w.P, w.L_cap, w.d), dtype=w.torch_dtype, pin_memory=True)
     Vh = torch.empty_like(Kh, pin_memory=True)
     Kd, Vd = synth.make_kv(w, device=dev)
@@ -500,18 +503,17 @@ def e2e_measure(w: synth.Workload, dev, stream, steps: int):
     out_h = torch.empty((w.P, w.G, w.d), dtype=torch.float32, pin_memory=True)
     sel_h = torch.empty((w.P, w.B), dtype=torch.int32, pin_memory=True)
     cnt_h = torch.empty((w.P,), dtype=torch.int32, pin_memory=True)
-    h2d = (Kh.numel() + Vh.numel() + qh.numel()) * Kh.element_size()
+    h2d = (2 * w.P * w.L * w.d + qh.numel()) * Kh.element_size()  # rows [0, L) of K, V; q
     d2h = out_h.numel() * 4 + sel_h.numel() * 4 + cnt_h.numel() * 4
+    copy_stream = torch.cuda.Stream(device=dev)
     times = []
     with torch.cuda.stream(stream):
         for i in range(steps + 1):
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            Kd.copy_(Kh, non_blocking=True)
-            Vd.copy_(Vh, non_blocking=True)
             qd.copy_(qh, non_blocking=True)
-            st.prefill(Kd, w.L, w.W, w.C, w.T)
+            st.prefill_from_host(Kh, Vh, Kd, Vd, w.L, w.W, w.C, w.T, copy_stream)
             st.step(qd, Kd, Vd)
             out_h.copy_(st.out, non_blocking=True)
             sel_h.copy_(st.sel_idx[:, :w.B], non_blocking=True)

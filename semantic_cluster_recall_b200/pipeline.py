@@ -95,6 +95,52 @@ class ClusterRecall:
             self.tail_begin.fill_(te)
             self.tail_end.fill_(L)
 
+    def prefill_from_host(self, K_host: torch.Tensor, V_host: torch.Tensor, K: torch.Tensor,
+                          V: torch.Tensor, L: int, W: int, C: int, iters: int,
+                          copy_stream: torch.cuda.Stream, groups: int = 8):
+        """prefill() for K and V that start in pinned host memory: the problems
+        are uploaded in `groups` groups on copy_stream, and each group is
+        clustered on the main stream as soon as its keys have arrived, so the
+        host-to-device copy (the bound here) overlaps the clustering. Values
+        follow the keys (only decoding reads them); the main stream waits for
+        them before returning. Rows [0, L) of every problem are copied."""
+        P = self.P
+        groups = max(1, min(groups, P))
+        main = self._main()
+        tb, te = self.S, L - W
+        ws = self._ws_cluster(te - tb, C)
+        start = torch.cuda.Event()
+        start.record(main)
+        copy_stream.wait_event(start)  # after everything queued before this call
+        bounds = [P * g // groups for g in range(groups + 1)]
+        arrived = []
+        with torch.cuda.stream(copy_stream):
+            for g in range(groups):
+                a, b = bounds[g], bounds[g + 1]
+                K[a:b, :L].copy_(K_host[a:b, :L], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_stream)
+                arrived.append(ev)
+            V[:, :L].copy_(V_host[:, :L], non_blocking=True)
+            v_done = torch.cuda.Event()
+            v_done.record(copy_stream)
+        for g in range(groups):
+            a, b = bounds[g], bounds[g + 1]
+            if a == b:
+                continue
+            main.wait_event(arrived[g])
+            ckv.ckv_cluster(K[a:b], K.stride(0), tb, te, C, iters, 0, 0, self.C_cap,
+                            self.perm_cap, self.centroids[a:b], self.centroids_hat[a:b],
+                            self.centroids_lp[a:b], self.labels[a:b], self.sizes[a:b],
+                            self.offsets[a:b], self.perm[a:b], ws, P=b - a, d=self.d,
+                            stream=main)
+        main.wait_event(v_done)
+        self.n_clustered, self.C_used, self.tail_lo = te - tb, C, te
+        with torch.cuda.stream(main):
+            self.n_clusters.fill_(C)
+            self.tail_begin.fill_(te)
+            self.tail_end.fill_(L)
+
     def incremental(self, K: torch.Tensor, n_tok: int, C: int, iters: int):
         """Cluster the oldest n_tok tail tokens into C new clusters appended to
         the metadata; the tail then starts after them."""

@@ -13,6 +13,10 @@ fills and one in the background, must give bit-identical outputs at every
 step (the steps read only published clusters, and the kernels are
 deterministic) and bit-identical metadata at the end. The synchronous run is
 itself checked against the oracle elsewhere (the 32-layer decode loop test).
+
+Prefill from host memory overlaps the upload of one group of problems with
+the clustering of the previous ones; it must give the same metadata as the
+one-call clustering of the same keys already on the device.
 """
 import numpy as np
 import pytest
@@ -106,3 +110,36 @@ def test_background_clustering_guards(cuda_device):
     torch.cuda.synchronize()
     assert int(st.n_clusters[0]) == w.C + w.inc_C
     assert ckv.ckv_device_error() == 0
+
+
+def test_prefill_from_host_equals_prefill(cuda_device):
+    # uploading in groups on a copy stream, each group clustered as it lands,
+    # gives the same metadata as clustering the device copy in one call
+    dev = cuda_device
+    w = W_SMALL.replace(P=10)
+    K, V = synth.make_kv(w, device=dev)
+    Kh = K.cpu().pin_memory()
+    Vh = V.cpu().pin_memory()
+    tb, te = w.S, w.L - w.W
+    n = te - tb
+    a = ClusterRecall(w.P, w.G, w.d, w.torch_dtype, w.L_cap, w.S, w.B, w.C, n, w.W, dev)
+    a.prefill(K, w.L, w.W, w.C, w.T)
+    Kd = torch.zeros_like(K)
+    Vd = torch.zeros_like(V)
+    main = torch.cuda.Stream(device=dev)
+    b = ClusterRecall(w.P, w.G, w.d, w.torch_dtype, w.L_cap, w.S, w.B, w.C, n, w.W, dev,
+                      stream=main)
+    with torch.cuda.stream(main):
+        b.prefill_from_host(Kh, Vh, Kd, Vd, w.L, w.W, w.C, w.T, torch.cuda.Stream(device=dev),
+                            groups=3)
+    torch.cuda.synchronize()
+    assert torch.equal(Kd[:, :w.L], K[:, :w.L]) and torch.equal(Vd[:, :w.L], V[:, :w.L])
+    for name in ("labels", "sizes", "offsets", "perm", "centroids", "centroids_hat",
+                 "centroids_lp", "n_clusters", "tail_begin", "tail_end"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    q = synth.make_queries(w, device=dev)
+    out_a = a.step(q, K, V)
+    with torch.cuda.stream(main):
+        out_b = b.step(q, Kd, Vd)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, out_b)
