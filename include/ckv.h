@@ -266,8 +266,11 @@ ckv_status ckv_select(const void *q, ckv_dtype dt, int P, int G, int d,
  * with the same arguments, outputs and results (sel_idx / sel_cnt
  * bit-identical to ckv_select; out equal to ckv_sparse_decode up to fp32
  * summation order). One thread-block cluster of up to 8 CTAs per problem
- * shares the scores, ranks and partial attention results through
- * distributed shared memory, so no workspace and no second kernel are
+ * (as many as keep every problem resident in one wave; one when even that
+ * needs several waves) shares the cluster scores and the partial attention
+ * results through distributed shared memory; each CTA finds the selection
+ * on its own copy of the scores (a weighted radix select for the cluster
+ * where the budget is reached), so no workspace and no second kernel are
  * needed. Supports G in {1, 2, 4} and up to 32768 attended rows per problem
  * (sink + budget + max_tail); other shapes return CKV_ERR_UNSUPPORTED (use
  * the two separate calls). */
