@@ -177,3 +177,38 @@ def test_tiny_f32_end_to_end(cuda_device):
             break
         assert centroid_rel_err(f32np(st.centroids[0, :w.C]), r["mu"]).max() <= CENT_REL_L2
         assert np.array_equal(st.perm[0, :n].cpu().numpy(), r["perm"])
+
+
+@pytest.mark.parametrize("metric", ["ip", "l2"])
+def test_full_size_assign_by_similarity(cuda_device, metric):
+    # the bench's assign_by_similarity launches (seeding + one assignment round
+    # of the bench workload under the distance ablation): seeds bit-exact on
+    # every problem, sampled tokens of sampled problems against the oracle
+    dev = cuda_device
+    w = synth.WORKLOADS["llama2_layer_32k"]
+    P, C, d = w.P, w.C, w.d
+    tb, te = w.S, w.L - w.W
+    n = te - tb
+    K, _ = synth.make_kv(w, device=dev, rows=w.L)
+    cent = torch.zeros((P, C, d), device=dev)
+    hat = torch.zeros((P, C, d), dtype=w.torch_dtype, device=dev)
+    lp = torch.zeros_like(hat)
+    bias = torch.zeros((P, C), device=dev)
+    labels = torch.full((P, n), -1, dtype=torch.int32, device=dev)
+    ckv.ckv_init_centroids_ex(K, K.stride(0), tb, te, C, 0, C, cent, hat, lp, metric=metric,
+                              bias=bias)
+    ckv.ckv_assign_ex(K, K.stride(0), tb, te, hat, C, 0, C, labels, 0, n,
+                      bias=bias if metric == "l2" else None)
+    torch.cuda.synchronize()
+    assert ckv.ckv_device_error() == 0
+    rng = np.random.default_rng(w.seed + 7)
+    lab = labels.cpu().numpy()
+    hat_h = hat.float().cpu().numpy().astype(np.float64)
+    for p in rng.choice(P, 3, replace=False):
+        kh = f32np(K[p, tb:te])
+        _, mh = oracle.init(kh, C, w.dtype, metric=metric)
+        assert np.array_equal(hat_h[p], mh)
+        toks = np.sort(rng.choice(n, SAMPLED_TOKENS, replace=False))
+        ref, gap = oracle.assign(kh[toks], mh, metric=metric)
+        bad = (lab[p, toks] != ref) & (gap >= GAP_EXEMPT)
+        assert not bad.any(), f"{metric} p={p}: {bad.sum()} non-tie differences"
