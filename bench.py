@@ -660,6 +660,15 @@ def run_ours(args):
         "gpu_launches": launches,
         "device_error_flags": err,
     }
+    if dec32 and "layer_loop" in dec32 and w.name == "llama2_layer_32k":
+        # the same step shape (32 KV heads, 32k context, C = 400, B = 1024) as
+        # many steps in one graph over rotated inputs (the 32 layers): no launch
+        # gap per step, and every step's data cold in L2
+        ll = dec32["layer_loop"]["per_layer_P32"]
+        line["decode"]["rotated_graph"] = {
+            "us_per_step": ll["us_per_step"], "steps_per_s": ll["steps_per_s"],
+            "roofline": ll["roofline"],
+            "launch": "32 fused launches (one per layer of the 32-layer workload) in one graph"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     line["clocks"] = clk.summary()
