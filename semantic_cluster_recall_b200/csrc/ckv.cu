@@ -85,6 +85,10 @@ enum { SLOT_ASSIGN_F32 = 0, SLOT_ASSIGN_BF16, SLOT_HIST, SLOT_SCATTER, SLOT_RANK
 
 bool valid_dtype(ckv_dtype dt) { return dt == CKV_F32 || dt == CKV_BF16; }
 
+#ifndef CKV_SD_PDL
+#define CKV_SD_PDL 1  // fused steps launched as programmatic dependents
+#endif
+
 bool valid_metric(int m) { return m == CKV_COSINE || m == CKV_INNER || m == CKV_L2; }
 
 int nchunks_of(int n) { return (n + IDX_CHUNK - 1) / IDX_CHUNK; }
@@ -691,13 +695,15 @@ ckv_status ckv_select_decode_cached(const void *q, ckv_dtype dt, int P, int G, i
     cfg.blockDim = dim3(sd::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = S(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = nc;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = CKV_SD_PDL;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = sd_optin(kern, smem);
     if (e == cudaSuccess) {
         void *args[] = {&a};

@@ -108,6 +108,13 @@ __host__ __device__ inline Layout layout(int C_cap, int G, int chunk, int nc) {
 template <typename T, int G, int U>
 __global__ void __launch_bounds__(THREADS)
 k_select_decode(const Args a) {
+    // programmatic dependent launch: wait for the preceding kernel of the
+    // stream before reading anything (its outputs may be this step's inputs),
+    // then let the next kernel be launched at once, so its CTAs are placed
+    // while this grid finishes (the gap between back-to-back steps). Both are
+    // no-ops when the launch carries no such dependency.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     cg::cluster_group cl = cg::this_cluster();
     const int nc = (int)cl.num_blocks();
     const int rank = (int)cl.block_rank();
