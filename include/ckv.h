@@ -374,6 +374,14 @@ ckv_status ckv_append(void *K, void *V, ckv_dtype dt, int P, int d, int64_t kv_p
                       int kv_rows, const void *new_k, const void *new_v, int32_t *tail_end,
                       void *stream);
 
+/* Self-test of the device timeout reporting (no counterpart in the paper):
+ * one thread waits, up to limit_us microseconds of the GPU's global timer, for
+ * a device flag that nothing sets, then records CKV_DEVERR_TIMEOUT in the
+ * device error word, exactly as a bounded wait inside a kernel does when it
+ * gives up. ckv_device_error then returns CKV_ERR_TIMEOUT; the context stays
+ * usable. limit_us in [0, 1000000]; CKV_ERR_INVALID otherwise. */
+ckv_status ckv_selftest_timeout(unsigned int limit_us, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

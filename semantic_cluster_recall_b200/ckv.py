@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(HERE, "libckv.so")
 CKV_OK, CKV_ERR_INVALID, CKV_ERR_CUDA, CKV_ERR_TIMEOUT, CKV_ERR_UNSUPPORTED = range(5)
 CKV_F32, CKV_BF16 = 0, 1
 CKV_DEVERR_LABEL, CKV_DEVERR_PERM, CKV_DEVERR_INDEX, CKV_DEVERR_OFFSETS = 1, 2, 4, 8
+CKV_DEVERR_TIMEOUT = 0x10
 MAX_CLUSTERS = 4096
 
 # every entry point declared in include/ckv.h
@@ -32,6 +33,7 @@ EXPORTS = [
     "ckv_sparse_decode_noalloc_scratch_bytes", "ckv_sparse_decode_noalloc",
     "ckv_select_decode", "ckv_cluster_ex", "ckv_cluster_ex_workspace_bytes",
     "ckv_init_centroids_ex", "ckv_assign_ex", "ckv_update_ex", "ckv_select_decode_cached",
+    "ckv_selftest_timeout",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -100,6 +102,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "ckv_select_decode_cached": (i32, [vp, i32, i32, i32, i32, vp, vp, i32, vp, vp, i32, i32,
                                            vp, vp, vp, vp, i64, i32, i32, vp, vp, i32, f32, vp,
                                            vp, i32, i32, vp, vp, vp]),
+        "ckv_selftest_timeout": (i32, [ctypes.c_uint, vp]),
         "ckv_sparse_decode_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, vp,
                                             vp, i32, vp, vp, i32, f32, vp, vp]),
     }
@@ -287,6 +290,12 @@ def ckv_select_decode(q, centroids_lp, n_clusters, C_cap, offsets, perm, perm_ca
                                   kv_rows, sink, _p(tail_begin), _p(tail_end), max_tail,
                                   float(scale), _p(out), _stream(stream))
     _check(st, "ckv_select_decode")
+
+
+def ckv_selftest_timeout(limit_us: int, stream=None):
+    """Make one bounded device wait give up (a flag nothing sets); the next
+    ckv_device_error reports the timeout."""
+    _check(load().ckv_selftest_timeout(int(limit_us), _stream(stream)), "ckv_selftest_timeout")
 
 
 NEVER_SELECTED = -(1 << 30)  # last-selected step of a cluster no step selected

@@ -806,6 +806,12 @@ ckv_status ckv_append(void *K, void *V, ckv_dtype dt, int P, int d, int64_t kv_p
     return launched("k_append");
 }
 
+ckv_status ckv_selftest_timeout(unsigned int limit_us, void *stream) {
+    if (limit_us > 1000000u) return fail(CKV_ERR_INVALID, "limit_us must be <= 1000000");
+    k_selftest_wait<<<1, 32, 0, S(stream)>>>((unsigned long long)limit_us * 1000ull);
+    return launched("k_selftest_wait");
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

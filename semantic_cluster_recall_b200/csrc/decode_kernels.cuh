@@ -206,4 +206,23 @@ k_append(T *__restrict__ K, T *__restrict__ V, int64_t kvs, int kv_rows,
     if (lane == 0) tail_end[p] = pos + 1;
 }
 
+// ---------------------------------------------------------------------------
+// Self-test of the timeout reporting: wait (bounded by the global timer) for a
+// flag that nothing sets, then record a timeout in the device error word.
+// ---------------------------------------------------------------------------
+__device__ int g_selftest_flag;  // never set
+
+__global__ void k_selftest_wait(unsigned long long limit_ns) {
+    if (threadIdx.x != 0) return;
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    while (*reinterpret_cast<volatile int *>(&g_selftest_flag) == 0) {
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > limit_ns) {
+            dev_flag(CKV_DEVERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
 }  // namespace ckv

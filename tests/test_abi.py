@@ -109,6 +109,8 @@ def test_validation_rejects_bad_arguments_without_launching(lib):
                                               fake, fake, fake, 2, None, None))
     _expect_invalid(lib.ckv_update_ex(fake, 1, 2, 128 * 100, 128, 0, 100, 4, 0, 8, fake, fake,
                                       100, fake, fake, fake, fake, 2, None, None))
+    # timeout self-test: a bound above one second
+    _expect_invalid(lib.ckv_selftest_timeout(2_000_000, None))
     # unknown dtype
     _expect_invalid(lib.ckv_assign(fake, 7, 2, 128 * 100, 128, 0, 100, fake, 4, 0, 8, fake, 0,
                                    100, None))
