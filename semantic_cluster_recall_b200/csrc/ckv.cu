@@ -566,7 +566,7 @@ ckv_status ckv_select(const void *q, ckv_dtype dt, int P, int G, int d, const vo
 #undef CKV_SCORE
     ckv_status s = launched("k_score");
     if (s) return s;
-    const size_t smem = (size_t)C_cap * 16;
+    const size_t smem = (size_t)C_cap * 36;
     cudaError_t e = smem_optin(k_rankfill, smem, SLOT_RANK);
     if (e != cudaSuccess) return fail(CKV_ERR_CUDA, "smem opt-in: %s", cudaGetErrorString(e));
     k_rankfill<<<P, 1024, smem, st>>>(scores, n_clusters, C_cap, offsets, perm, perm_cap, budget,
